@@ -1,0 +1,471 @@
+"""Benchmark: MoE dispatch + combine (forward and backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--fwd-only] [--no-e2e] [--no-cpu-baseline]
+
+A step is one pass of the whole path over one batch of the DeepSeek-V3-shaped
+decode workload (T=4096 tokens, H=7168, E=256 experts, K=8, 8 logical EP
+ranks, Zipf(0.6) routing):
+    layout -> permute (bf16, with chunk-completion counters) -> combine
+    (identity experts: y = the dispatched rows) -> combine backward ->
+    dispatch backward.
+value = algorithmic HBM bytes of the step / device time of the step, in GB/s
+(also reported: tokens/s).  Inputs are resident in HBM when the timed region
+starts; L2 is flushed (256 MiB write) before every timed step and the flush
+is outside the timed events.  With N GPUs (torchrun), every rank runs its own
+replica on its own data (weak scaling; no collective on the data path); the
+reported time is the max over ranks.
+
+--impl reference times the CPU oracle (single-threaded C) on a bounded sample
+of the same workload and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import glob
+import hashlib
+import io
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine HBM GB/s and tokens/s on 1 B200; fraction of HBM peak"
+CONFIG_INDEX = 2
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--fwd-only", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- bytes --
+def step_bytes(T, K, H, E, P, fwd_only=False):
+    """Algorithmic bytes per call (what the method must move at least)."""
+    TK = T * K
+    b = {
+        "layout": 4 * TK + 4 * TK + 4 * P + 8 * E,
+        "permute": 2 * T * H + 2 * P * H,
+        "combine": 2 * TK * H + 8 * TK + 2 * T * H,
+    }
+    if not fwd_only:
+        b["combine_bwd"] = 2 * T * H + 2 * TK * H + 2 * P * H + 12 * TK
+        b["dispatch_bwd"] = 2 * TK * H + 2 * T * H + 4 * TK
+    return b
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic(kernel_key: str):
+    """dram bytes per launch of `kernel_key` from the committed ncu summaries,
+    if the kernel's source file is unchanged since the capture (else None).
+    Summary lines look like:  traffic: <key> <bytes per launch> src=<sha1[:12]>"""
+    srcfile = {"permute": "permute.cu", "combine": "combine.cu", "combine_bwd": "combine.cu",
+               "dispatch_bwd": "combine.cu", "layout": "layout.cu"}.get(kernel_key)
+    if srcfile is None:
+        return None
+    src = os.path.join(ROOT, "combine_moe_dispatch_05_b200", "csrc", srcfile)
+    try:
+        sha = hashlib.sha1(open(src, "rb").read()).hexdigest()[:12]
+    except OSError:
+        return None
+    for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(f):
+            m = re.match(r"\s*traffic:\s+(\S+)\s+(\d+)\s+src=([0-9a-f]+)", line)
+            if m and m.group(1) == kernel_key and m.group(3) == sha:
+                return int(m.group(2))
+    return None
+
+
+# ---------------------------------------------------------------- clocks --
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: str):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        for r in csv.reader(io.StringIO(self.out or "")):
+            if len(r) < 9:
+                continue
+            try:
+                rows.append((float(r[1]), float(r[2]), float(r[3]), [x.strip() for x in r[4:9]]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3][1:])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows),
+                "samples": len(rows), "samples_under_load": len(loaded),
+                "reasons": reasons}
+
+
+def smi_id(torch, dev) -> str:
+    """nvidia-smi --id for a torch device: its PCI bus id when torch exposes it
+    (robust to CUDA_VISIBLE_DEVICES remapping), else the ordinal."""
+    p = torch.cuda.get_device_properties(dev)
+    try:
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except AttributeError:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[dev.index].strip()
+        return str(dev.index)
+
+
+# ------------------------------------------------------ distributed glue --
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each replica draws its own batch (weak scaling)."""
+    return rank
+
+
+# ------------------------------------------------------------- our arm --
+def run_ours(args, world, rank, local):
+    import torch
+    from combine_moe_dispatch_05_b200 import ops
+    from combine_moe_dispatch_05_b200 import workloads as W
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ops.lib()  # fails loudly if the CUDA library is missing
+    s = W.config(CONFIG_INDEX, rank_seed_offset(rank))
+    T, H, E, K, R = s.T, s.H, s.E, s.K, s.R
+
+    ids_h = W.topk_ids(s).pin_memory()
+    sc_h = W.topk_scales(s).pin_memory()
+    x_h = W.tokens(s).pin_memory()
+    g_h = W.grad_out(s).pin_memory()
+    ids, sc, x, g = (t.to(dev) for t in (ids_h, sc_h, x_h, g_h))
+
+    L = ops.alloc_layout(T, K, E, R, dev)
+    P_cap = L.P_cap
+    xp = torch.empty((P_cap, H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    gy = torch.empty((P_cap, H), dtype=torch.bfloat16, device=dev)
+    gs = torch.empty((T, K), dtype=torch.float32, device=dev)
+    gx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    st = ops.new_status(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        rec = (lambda i: evs[i].record(stream)) if evs else (lambda i: None)
+        rec(0)
+        ops.moe_dispatch_layout(ids, E, R, layout=L, status=st)
+        rec(1)
+        ops.moe_dispatch_permute(x, L, xp=xp, status=st)
+        rec(2)
+        ops.moe_combine(xp, L.dst_row, sc, out=out, status=st)   # identity experts: y = xp
+        rec(3)
+        if not args.fwd_only:
+            ops.moe_combine_bwd(g, xp, sc, L, grad_y=gy, grad_scales=gs, status=st)
+            rec(4)
+            ops.moe_dispatch_bwd(gy, L.dst_row, T, K, grad_x=gx, status=st)
+            rec(5)
+
+    phases = ["layout", "permute", "combine"] + ([] if args.fwd_only else
+                                                 ["combine_bwd", "dispatch_bwd"])
+    n_ev = len(phases) + 1
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if ops.read_status(st) != 0:
+        raise RuntimeError(f"device status {ops.read_status(st)}")
+    P = int(L.expert_offsets[E].item())
+    nbytes = step_bytes(T, K, H, E, P, args.fwd_only)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(smi_id(torch, dev)) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    per_phase = {p: [] for p in phases}
+    step_ms = []
+    for e in evs:
+        step_ms.append(e[0].elapsed_time(e[-1]))
+        for j, p in enumerate(phases):
+            per_phase[p].append(e[j].elapsed_time(e[j + 1]))
+    total_ms = sum(step_ms)
+    total_ms_max = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms_max / args.steps
+    bytes_step = sum(nbytes.values())
+    value = bytes_step * world / (ms_per_step * 1e-3) / 1e9
+    tok_s = T * world / (ms_per_step * 1e-3)
+
+    phase_us = {p: 1e3 * statistics.mean(v) for p, v in per_phase.items()}
+    phase_gbs = {p: nbytes[p] / (phase_us[p] * 1e-6) / 1e9 for p in phases}
+    dom = max((p for p in phases if p != "layout"), key=lambda p: phase_us[p])
+    peak, peak_src = measured_peak()
+    fwd_us = sum(phase_us[p] for p in ("layout", "permute", "combine"))
+    fwd_bytes = sum(nbytes[p] for p in ("layout", "permute", "combine"))
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(phase_gbs[dom], 1),
+                "peak": peak, "unit": "GB/s", "frac": round(phase_gbs[dom] / peak, 4),
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src ==
+                "measured" else "fallback 6.65 TB/s",
+                "traffic": ncu_traffic(dom),
+                "algorithmic_bytes_per_launch": nbytes[dom],
+                "step_frac": round(bytes_step / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+                "fwd_frac": round(fwd_bytes / (fwd_us * 1e-6) / 1e9 / peak, 4)}
+
+    res = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s",
+           "tokens_per_s": round(tok_s, 1), "n_gpus": world, "steps": args.steps,
+           "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 5),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded Zipf routing, N(0,1) activations; identity experts)",
+           "config": {"workload": f"{s.name}: T={T} H={H} E={E} K={K} R={R} Zipf(s={s.zipf_s})"
+                                  f" {'fwd' if args.fwd_only else 'fwd+bwd'}",
+                      "P": P, "P_cap": P_cap, "bytes_per_step": bytes_step,
+                      "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                      "parallelism": f"replicas x{world}"},
+           "phases_us": {p: round(v, 2) for p, v in phase_us.items()},
+           "phases_gbs": {p: round(v, 1) for p, v in phase_gbs.items()},
+           "roofline": roofline,
+           "gpu_launches": (7 if not args.fwd_only else 5) * args.steps,
+           "clocks": clk.summary()}
+
+    if not args.no_e2e:
+        res["e2e"] = e2e(args, ops, torch, dev, stream, L, (ids_h, sc_h, x_h, g_h),
+                         (ids, sc, x, g), (xp, out, gy, gs, gx, st), flush, T, K, E, R,
+                         bytes_step, world)
+    return res
+
+
+def e2e(args, ops, torch, dev, stream, L, host_in, dev_in, bufs, flush, T, K, E, R, bytes_step,
+        world):
+    """Same step through the public API with host buffers: H2D of the step's
+    inputs from pinned memory, the calls, D2H of the results, all timed."""
+    ids_h, sc_h, x_h, g_h = host_in
+    ids, sc, x, g = dev_in
+    xp, out, gy, gs, gx, st = bufs
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    gx_h = torch.empty(gx.shape, dtype=gx.dtype, pin_memory=True)
+    gs_h = torch.empty(gs.shape, dtype=gs.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = out.numel() * 2 + (0 if args.fwd_only else gx.numel() * 2 + gs.numel() * 4)
+
+    def one():
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        ops.moe_dispatch_layout(ids, E, R, layout=L, status=st)
+        ops.moe_dispatch_permute(x, L, xp=xp, status=st)
+        ops.moe_combine(xp, L.dst_row, sc, out=out, status=st)
+        out_h.copy_(out, non_blocking=True)
+        if not args.fwd_only:
+            ops.moe_combine_bwd(g, xp, sc, L, grad_y=gy, grad_scales=gs, status=st)
+            ops.moe_dispatch_bwd(gy, L.dst_row, T, K, grad_x=gx, status=st)
+            gx_h.copy_(gx, non_blocking=True)
+            gs_h.copy_(gs, non_blocking=True)
+
+    for _ in range(3):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        one()
+        b.record(stream)
+        b.synchronize()
+        tot += a.elapsed_time(b)
+    tot = max_over_ranks(tot, world)
+    ms = tot / args.steps
+    return {"value": round(bytes_step * world / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "ms_per_step": round(ms, 4), "tokens_per_s": round(T * world / (ms * 1e-3), 1),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# --------------------------------------------------------- oracle timing --
+def oracle_step_sample(T_sample: int, fwd_only: bool):
+    """One pass of the oracle over the first T_sample tokens of the workload.
+    Returns (seconds, algorithmic bytes of the sample)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from combine_moe_dispatch_05_b200 import workloads as W
+
+    s = W.config(CONFIG_INDEX)
+    ids = W.topk_ids(s)[:T_sample].numpy()
+    sc = W.topk_scales(s)[:T_sample].numpy()
+    x = W.as_u16(W.tokens(s.with_(T=T_sample)))
+    g = W.as_u16(W.grad_out(s.with_(T=T_sample)))
+    t0 = time.perf_counter()
+    L = oracle.layout(ids, s.E, s.R)
+    xp = np.zeros((L.P_cap, s.H), np.uint16)
+    oracle.permute_rows(x, L.dst_row, s.K, L.counts, L.offsets, xp)
+    oracle.combine(xp, L.dst_row, sc, None)
+    if not fwd_only:
+        gy = np.zeros_like(xp)
+        oracle.combine_bwd(g, xp, sc, L.dst_row, L.counts, L.offsets, gy)
+        oracle.dispatch_bwd(gy, L.dst_row, T_sample, s.K)
+    dt = time.perf_counter() - t0
+    b = sum(step_bytes(T_sample, s.K, s.H, s.E, L.P, fwd_only).values())
+    return dt, b, s
+
+
+ORACLE_SAMPLE_TOKENS = 1024
+
+
+def cpu_baseline(fwd_only):
+    dt, b, s = oracle_step_sample(ORACLE_SAMPLE_TOKENS, fwd_only)
+    return {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "seconds": round(dt, 3),
+            "tokens_per_s": round(ORACLE_SAMPLE_TOKENS / dt, 1),
+            "sample": f"first {ORACLE_SAMPLE_TOKENS} of the {s.T} tokens of the same workload, "
+                      f"one full {'fwd' if fwd_only else 'fwd+bwd'} pass of the single-threaded "
+                      f"C oracle"}
+
+
+REFERENCE_BUDGET_S = 150.0
+
+
+def run_reference(args):
+    """The oracle, as it stands, on the host: each step is one pass over a
+    token sample of the workload, sized so the whole run stays within about
+    REFERENCE_BUDGET_S seconds."""
+    from combine_moe_dispatch_05_b200 import workloads as W
+    s = W.config(CONFIG_INDEX)
+    probe_tokens = 64
+    dt, _, _ = oracle_step_sample(probe_tokens, args.fwd_only)      # untimed probe
+    per_token = dt / probe_tokens
+    n_steps = args.steps + max(0, args.warmup - 1)
+    sample = int(REFERENCE_BUDGET_S / max(n_steps, 1) / per_token)
+    sample = max(16, min(ORACLE_SAMPLE_TOKENS, sample))
+    for _ in range(max(0, args.warmup - 1)):
+        oracle_step_sample(sample, args.fwd_only)
+    tot, tot_b = 0.0, 0
+    for _ in range(args.steps):
+        dt, b, _ = oracle_step_sample(sample, args.fwd_only)
+        tot += dt
+        tot_b += b
+    v = tot_b / tot / 1e9
+    ms = 1e3 * tot / args.steps
+    desc = (f"first {sample} of the {s.T} tokens per step, single-threaded C oracle, "
+            f"{'fwd' if args.fwd_only else 'fwd+bwd'}")
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "GB/s",
+            "tokens_per_s": round(sample / (ms * 1e-3), 1), "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"{s.name}: T={s.T} H={s.H} E={s.E} K={s.K} R={s.R} "
+                                   f"Zipf(s={s.zipf_s}) {'fwd' if args.fwd_only else 'fwd+bwd'}",
+                       "sample_tokens": sample},
+            "cpu_baseline": {"value": round(v, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(v, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        res = run_ours(args, world, rank, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(args.fwd_only)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,385 @@
+// Combine and the two backward calls.
+//
+// Combine is defined by the torch_npu "npu_moe_distribute_combine" API
+// reference (function description): the expert outputs are brought back along
+// the dispatch path, multiplied by their expert_scales and summed, and the
+// shared-expert output is added without a weight (parameter expert_scales).
+// Here the "way back" is the dispatch map itself: out[t] gathers the K rows
+// dst_row[t*K + k] of the expert-major buffer.
+//
+// combine_bwd and dispatch_bwd are the adjoints of the two linear maps
+// (combine in y and in the scales; permute = copy of x[t] to K rows).
+//
+// B200 design.  All three are HBM-bound gathers / scatters of 16-byte
+// vectors; there is no contraction to put on tensor cores.
+//   * combine / dispatch_bwd: a warp owns a unit = (token, 64-vector column
+//     chunk); lanes 0..K-1 fetch the slot's row index and scale once and
+//     broadcast them with shuffles; every lane then issues all K 16-byte
+//     gathers of its two columns before reducing, so each warp keeps up to
+//     2*K*512 bytes of loads in flight.  The fp32 reduction runs k = 0..K-1
+//     in order with fma, then adds the shared row, then rounds once.
+//   * combine_bwd: a 256-thread CTA owns a token row: it reads grad_out[t]
+//     once, gathers the K rows of y, writes the K scaled rows of grad_y and
+//     reduces the K dot products across the CTA in a fixed order
+//     (deterministic).  The same CTAs then zero the padding rows of grad_y.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kGatherThreads = 256;
+constexpr int kVecPerLane = 2;   // 16-byte columns per lane per unit
+constexpr int kKBatch = 8;       // gathers issued before reducing
+
+template <bool kScaled, bool kShared>
+__global__ void __launch_bounds__(kGatherThreads)
+gather_reduce_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ dst_row,
+                     const float* __restrict__ scales, const uint16_t* __restrict__ shared,
+                     int64_t T, int K, int H, int64_t P_cap, uint16_t* __restrict__ out,
+                     int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_id = ((int64_t)blockIdx.x * kGatherThreads + threadIdx.x) >> 5;
+  const int64_t n_warps = ((int64_t)gridDim.x * kGatherThreads) >> 5;
+  const int V = H >> 3;
+  constexpr int kUnitVecs = 32 * kVecPerLane;
+  const int units_per_token = (V + kUnitVecs - 1) / kUnitVecs;
+  const int64_t n_units = T * units_per_token;
+
+  for (int64_t u = warp_id; u < n_units; u += n_warps) {
+    const int64_t t = u / units_per_token;
+    const int c = (int)(u - t * units_per_token);
+
+    int my_row = -1;
+    float my_s = 1.0f;
+    if (lane < K) {
+      my_row = __ldg(dst_row + t * K + lane);
+      if (kScaled) my_s = __ldg(scales + t * K + lane);
+      if (my_row != -1 && (my_row < 0 || (int64_t)my_row >= P_cap)) {
+        record_error(status, MOE_ERR_BOUNDS);
+        my_row = -1;
+      }
+    }
+
+    float acc[kVecPerLane][8];
+#pragma unroll
+    for (int i = 0; i < kVecPerLane; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
+
+    for (int kb = 0; kb < K; kb += kKBatch) {
+      int rows[kKBatch];
+      uint4 v[kKBatch][kVecPerLane];
+#pragma unroll
+      for (int j = 0; j < kKBatch; ++j) {
+        rows[j] = __shfl_sync(0xffffffffu, my_row, (kb + j) & 31);
+        if (kb + j >= K) rows[j] = -1;
+#pragma unroll
+        for (int i = 0; i < kVecPerLane; ++i) {
+          const int vec = c * kUnitVecs + i * 32 + lane;
+          if (rows[j] >= 0 && vec < V)
+            v[j][i] = ld_nc_v4(y + (int64_t)rows[j] * H + (int64_t)vec * 8);
+          else
+            v[j][i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kKBatch; ++j) {
+        const float s = __shfl_sync(0xffffffffu, my_s, (kb + j) & 31);
+        if (rows[j] < 0) continue;  // an unplaced slot contributes nothing
+#pragma unroll
+        for (int i = 0; i < kVecPerLane; ++i) {
+          const uint32_t w[4] = {v[j][i].x, v[j][i].y, v[j][i].z, v[j][i].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (kScaled) {
+              acc[i][2 * q] = fmaf(s, bf16_lo(w[q]), acc[i][2 * q]);
+              acc[i][2 * q + 1] = fmaf(s, bf16_hi(w[q]), acc[i][2 * q + 1]);
+            } else {
+              acc[i][2 * q] = __fadd_rn(acc[i][2 * q], bf16_lo(w[q]));
+              acc[i][2 * q + 1] = __fadd_rn(acc[i][2 * q + 1], bf16_hi(w[q]));
+            }
+          }
+        }
+      }
+    }
+
+#pragma unroll
+    for (int i = 0; i < kVecPerLane; ++i) {
+      const int vec = c * kUnitVecs + i * 32 + lane;
+      if (vec >= V) continue;
+      if (kShared) {
+        const uint4 sv = ld_nc_v4(shared + t * H + (int64_t)vec * 8);
+        const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[i][2 * q] = __fadd_rn(acc[i][2 * q], bf16_lo(w[q]));
+          acc[i][2 * q + 1] = __fadd_rn(acc[i][2 * q + 1], bf16_hi(w[q]));
+        }
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[i][0], acc[i][1]);
+      o.y = pack_bf16x2(acc[i][2], acc[i][3]);
+      o.z = pack_bf16x2(acc[i][4], acc[i][5]);
+      o.w = pack_bf16x2(acc[i][6], acc[i][7]);
+      st_v4(out + t * H + (int64_t)vec * 8, o);
+    }
+  }
+}
+
+constexpr int kBwdThreads = 256;
+constexpr int kBwdWarps = kBwdThreads / 32;
+
+__global__ void __launch_bounds__(kBwdThreads)
+combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ y,
+                   const float* __restrict__ scales, const int32_t* __restrict__ dst_row,
+                   const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
+                   int E, int64_t T, int K, int H, int64_t P_cap,
+                   uint16_t* __restrict__ grad_y, float* __restrict__ grad_s,
+                   int32_t* status) {
+  __shared__ int32_t s_row[MOE_MAX_TOPK];
+  __shared__ float s_sc[MOE_MAX_TOPK];
+  __shared__ float s_part[kBwdWarps][MOE_MAX_TOPK];
+  __shared__ int32_t s_padpref[MOE_MAX_EXPERTS + 1];
+  __shared__ int32_t s_pad_base[MOE_MAX_EXPERTS];
+  __shared__ int32_t s_warp[kBwdWarps];
+  __shared__ int s_bad;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int V = H >> 3;
+
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    if (tid < K) {
+      int r = __ldg(dst_row + t * K + tid);
+      if (r != -1 && (r < 0 || (int64_t)r >= P_cap)) {
+        record_error(status, MOE_ERR_BOUNDS);
+        r = -1;
+      }
+      s_row[tid] = r;
+      s_sc[tid] = __ldg(scales + t * K + tid);
+    }
+    __syncthreads();
+
+    float dot[MOE_MAX_TOPK];
+#pragma unroll
+    for (int k = 0; k < MOE_MAX_TOPK; ++k) dot[k] = 0.0f;
+
+    for (int vec = tid; vec < V; vec += kBwdThreads) {
+      const uint4 gv = ld_nc_v4(g + t * H + (int64_t)vec * 8);
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+      float gf[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        gf[2 * q] = bf16_lo(gw[q]);
+        gf[2 * q + 1] = bf16_hi(gw[q]);
+      }
+#pragma unroll
+      for (int kb = 0; kb < MOE_MAX_TOPK; kb += kKBatch) {
+        if (kb >= K) break;
+        uint4 yv[kKBatch];
+#pragma unroll
+        for (int j = 0; j < kKBatch; ++j) {
+          const int k = kb + j;
+          const int r = k < K ? s_row[k] : -1;
+          yv[j] = r >= 0 ? ld_nc_v4(y + (int64_t)r * H + (int64_t)vec * 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < kKBatch; ++j) {
+          const int k = kb + j;
+          const int r = k < K ? s_row[k] : -1;
+          if (r < 0) continue;
+          const float s = s_sc[k];
+          const uint32_t yw[4] = {yv[j].x, yv[j].y, yv[j].z, yv[j].w};
+          float d = dot[k];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            d = fmaf(gf[2 * q], bf16_lo(yw[q]), d);
+            d = fmaf(gf[2 * q + 1], bf16_hi(yw[q]), d);
+          }
+          dot[k] = d;
+          uint4 o;
+          o.x = pack_bf16x2(__fmul_rn(s, gf[0]), __fmul_rn(s, gf[1]));
+          o.y = pack_bf16x2(__fmul_rn(s, gf[2]), __fmul_rn(s, gf[3]));
+          o.z = pack_bf16x2(__fmul_rn(s, gf[4]), __fmul_rn(s, gf[5]));
+          o.w = pack_bf16x2(__fmul_rn(s, gf[6]), __fmul_rn(s, gf[7]));
+          st_v4(grad_y + (int64_t)r * H + (int64_t)vec * 8, o);
+        }
+      }
+    }
+
+    // fixed-order reduction of the K dot products over the CTA
+#pragma unroll
+    for (int k = 0; k < MOE_MAX_TOPK; ++k) {
+      if (k >= K) break;
+      float d = dot[k];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      if (lane == 0) s_part[warp][k] = d;
+    }
+    __syncthreads();
+    if (tid < K) {
+      float sum = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kBwdWarps; ++w) sum += s_part[w][tid];
+      grad_s[t * K + tid] = s_row[tid] >= 0 ? sum : 0.0f;
+    }
+    __syncthreads();
+  }
+
+  // ---- zero the padding rows (below P) of grad_y ----
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  for (int e = tid; e < E; e += kBwdThreads) {
+    const int c = __ldg(counts + e);
+    const int pad = (__ldg(offsets + e + 1) - __ldg(offsets + e)) - c;
+    if (pad < 0 || pad >= kTile || c < 0) s_bad = 1;
+    s_pad_base[e] = __ldg(offsets + e) + c;
+  }
+  // exclusive prefix of the padding counts (E <= 512: two per thread)
+  {
+    int p[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int e = 2 * tid + i;
+      p[i] = 0;
+      if (e < E) {
+        const int c = __ldg(counts + e);
+        const int pad = (__ldg(offsets + e + 1) - __ldg(offsets + e)) - c;
+        p[i] = (pad >= 0 && pad < kTile) ? pad : 0;
+      }
+    }
+    const int local = p[0] + p[1];
+    const int incl = warp_inclusive_scan(local);
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int v = lane < kBwdWarps ? s_warp[lane] : 0;
+      const int wi = warp_inclusive_scan(v);
+      if (lane < kBwdWarps) s_warp[lane] = wi - v;
+    }
+    __syncthreads();
+    const int excl = s_warp[warp] + incl - local;
+    if (2 * tid < E) s_padpref[2 * tid] = excl;
+    if (2 * tid + 1 < E) s_padpref[2 * tid + 1] = excl + p[0];
+    if (2 * tid == E - 1 || 2 * tid + 1 == E - 1) s_padpref[E] = excl + local;
+    __syncthreads();
+  }
+  if (s_bad || (int64_t)__ldg(offsets + E) > P_cap) {
+    if (tid == 0) record_error(status, MOE_ERR_BOUNDS);
+    return;
+  }
+  const int pad_total = s_padpref[E];
+  for (int q = blockIdx.x; q < pad_total; q += gridDim.x) {
+    int lo = 0, hi = E - 1;  // last expert with padpref <= q
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_padpref[mid] <= q) lo = mid; else hi = mid - 1;
+    }
+    const int64_t r = (int64_t)s_pad_base[lo] + (q - s_padpref[lo]);
+    for (int vec = tid; vec < V; vec += kBwdThreads)
+      st_v4(grad_y + r * H + (int64_t)vec * 8, make_uint4(0, 0, 0, 0));
+  }
+}
+
+// Blocks per SM for a kernel, cached per device.
+template <typename F>
+int blocks_per_sm(F kernel, int threads, int device, int* cache) {
+  if (device >= 0 && device < 64 && cache[device] > 0) return cache[device];
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1)
+    n = 1;
+  if (device >= 0 && device < 64) cache[device] = n;
+  return n;
+}
+
+int g_occ_comb[4][64];
+int g_occ_bwd[64];
+
+template <bool kScaled, bool kShared>
+int launch_gather(int slot, const uint16_t* y, const int32_t* dst_row, const float* scales,
+                  const uint16_t* shared, int64_t T, int K, int H, int64_t P_cap, uint16_t* out,
+                  int32_t* status, cudaStream_t s) {
+  const int dev = moe_host::current_device();
+  auto kern = gather_reduce_kernel<kScaled, kShared>;
+  const int bps = blocks_per_sm(kern, kGatherThreads, dev, g_occ_comb[slot]);
+  const int64_t units = T * (((H >> 3) + 63) / 64);
+  int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
+  const int64_t need = (units + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
+  if (grid > need) grid = need;
+  if (grid < 1) grid = 1;
+  kern<<<(unsigned)grid, kGatherThreads, 0, s>>>(y, dst_row, scales, shared, T, K, H, P_cap, out,
+                                                 status);
+  return moe_host::launch_status();
+}
+
+int check_rows_args(const void* y, const int32_t* dst_row, int64_t T, int K, int H,
+                    int64_t P_cap, const void* out) {
+  if (T < 0 || K < 1 || K > MOE_MAX_TOPK || H <= 0 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (T * (int64_t)K > (int64_t)INT32_MAX || P_cap < 0 || P_cap > (int64_t)INT32_MAX)
+    return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!y || !dst_row || !out)) return MOE_ERR_INVALID_ARG;
+  if ((y && !moe_host::aligned16(y)) || (out && !moe_host::aligned16(out)))
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_combine(const void* y, const int32_t* dst_row, const float* scales,
+                           const void* shared_x, int64_t T, int K, int H, int64_t P_cap,
+                           void* out, int32_t* d_status, void* stream) {
+  using namespace moe;
+  int st = check_rows_args(y, dst_row, T, K, H, P_cap, out);
+  if (st != MOE_OK) return st;
+  if (T > 0 && !scales) return MOE_ERR_INVALID_ARG;
+  if (shared_x && !moe_host::aligned16(shared_x)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t* yy = static_cast<const uint16_t*>(y);
+  uint16_t* o = static_cast<uint16_t*>(out);
+  if (shared_x)
+    return launch_gather<true, true>(0, yy, dst_row, scales,
+                                     static_cast<const uint16_t*>(shared_x), T, K, H, P_cap, o,
+                                     d_status, s);
+  return launch_gather<true, false>(1, yy, dst_row, scales, nullptr, T, K, H, P_cap, o,
+                                    d_status, s);
+}
+
+extern "C" int moe_dispatch_bwd(const void* grad_xp, const int32_t* dst_row, int64_t T, int K,
+                                int H, int64_t P_cap, void* grad_x, int32_t* d_status,
+                                void* stream) {
+  using namespace moe;
+  int st = check_rows_args(grad_xp, dst_row, T, K, H, P_cap, grad_x);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  return launch_gather<false, false>(2, static_cast<const uint16_t*>(grad_xp), dst_row, nullptr,
+                                     nullptr, T, K, H, P_cap, static_cast<uint16_t*>(grad_x),
+                                     d_status, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int moe_combine_bwd(const void* grad_out, const void* y, const float* scales,
+                               const int32_t* dst_row, const int32_t* expert_counts,
+                               const int32_t* expert_offsets, int E, int64_t T, int K, int H,
+                               int64_t P_cap, void* grad_y, float* grad_scales,
+                               int32_t* d_status, void* stream) {
+  using namespace moe;
+  int st = check_rows_args(y, dst_row, T, K, H, P_cap, grad_y);
+  if (st != MOE_OK) return st;
+  if (E < 1 || E > MOE_MAX_EXPERTS || !expert_counts || !expert_offsets || !grad_y)
+    return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!grad_out || !scales || !grad_scales)) return MOE_ERR_INVALID_ARG;
+  if (grad_out && !moe_host::aligned16(grad_out)) return MOE_ERR_INVALID_ARG;
+  if (!moe_host::aligned16(grad_y)) return MOE_ERR_INVALID_ARG;
+  if (P_cap < moe_padded_capacity(T, K, E)) return MOE_ERR_CAPACITY;
+  if (T == 0) return MOE_OK;  // P = 0: no rows to write
+  const int dev = moe_host::current_device();
+  const int bps = blocks_per_sm(combine_bwd_kernel, kBwdThreads, dev, g_occ_bwd);
+  int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
+  const int64_t need = T + (int64_t)(kTile - 1) * E;
+  if (grid > need) grid = need;
+  combine_bwd_kernel<<<(unsigned)grid, kBwdThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(grad_out), static_cast<const uint16_t*>(y), scales, dst_row,
+      expert_counts, expert_offsets, E, T, K, H, P_cap, static_cast<uint16_t*>(grad_y),
+      grad_scales, d_status);
+  return moe_host::launch_status();
+}

@@ -1,0 +1,352 @@
+// Dispatch permute: the "fused unzip" of the DeepEP pull request "Intra-node
+// compute compensation + overlap robustness (CUDA719 fix)" (Kernel / host),
+// for one GPU: every token row is scattered into its K expert rows of the
+// expert-major buffer (expand_x of the torch_npu npu_moe_distribute_combine
+// API), padding rows of each expert's last 128-row M-tile (TEMPO summary,
+// section 1) are zero-filled, and each finished row bumps its tile's
+// chunk-completion counter with atom.acq_rel.gpu.
+//
+// B200 design.  The work is pure data movement, so it is written as a bulk
+// copy engine rather than as threads moving registers:
+//   * one warp per CTA; lane 0 drives the SM's bulk-copy (TMA) unit: a
+//     non-multicast cp.async.bulk global -> shared load of each token row
+//     (or 16 KiB column chunk) into an S-stage ring, completed on an
+//     mbarrier, then K cp.async.bulk shared -> global stores of the same
+//     bytes, one per destination row.  The row is read from HBM once and
+//     never passes through registers.
+//   * padding rows are bulk-stored from a zero-filled shared chunk.
+//   * work is split by "virtual rows": the T*K slots followed by the
+//     padding rows, cut into equal contiguous ranges per CTA, so every CTA
+//     writes the same number of rows whatever the expert skew.
+//   * counters: a row's +1 is released only after its bulk-store group has
+//     completed (cp.async.bulk.wait_group), behind a proxy fence, with a lag
+//     of a few groups so the copy pipeline never drains.  FP8 scale rows are
+//     copied by the 32 lanes with plain stores before the same release.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr uint32_t kMaxChunk = 16384;  // bytes per bulk copy
+constexpr int kMaxStages = 16;
+constexpr int kRelLag = 2;             // bulk groups kept in flight before a release
+constexpr int kPermCtasPerSm = 2;
+
+struct PermArgs {
+  const uint8_t* x;
+  int64_t x_stride_bytes;
+  int64_t row_bytes;
+  const float* x_scales;
+  int64_t xs_stride;   // elements
+  int scale_cols;      // H/128 on the E4M3 path, 0 otherwise
+  const int32_t* dst_row;
+  int64_t T;
+  int K;
+  const int32_t* counts;
+  const int32_t* offsets;
+  int E;
+  uint8_t* xp;
+  float* xp_scales;
+  int64_t P_cap;
+  uint32_t* tile_ready;
+  int32_t* status;
+  uint32_t chunk_cap;   // bytes per chunk (multiple of 16)
+  uint32_t stage_bytes; // chunk_cap rounded up to 128
+  int n_chunks;
+  int stages;
+};
+
+__device__ __forceinline__ uint32_t chunk_len(const PermArgs& a, int ch) {
+  const int64_t rem = a.row_bytes - (int64_t)ch * a.chunk_cap;
+  return (uint32_t)(rem < (int64_t)a.chunk_cap ? rem : (int64_t)a.chunk_cap);
+}
+
+// Destination row of a slot, or -1 if it must be skipped (unplaced slot, or a
+// row outside the buffer, which is reported).
+__device__ __forceinline__ int64_t checked_row(const PermArgs& a, int64_t slot) {
+  const int32_t r = __ldg(a.dst_row + slot);
+  if (r == -1) return -1;
+  if (r < 0 || (int64_t)r >= a.P_cap) {
+    record_error(a.status, MOE_ERR_BOUNDS);
+    return -1;
+  }
+  return r;
+}
+
+__global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
+  __shared__ int32_t s_cnt[MOE_MAX_EXPERTS];
+  __shared__ int32_t s_padpref[MOE_MAX_EXPERTS + 1];
+
+  const int lane = threadIdx.x;
+  const int S = a.stages;
+  uint8_t* stage0 = smem;
+  uint8_t* zero = smem + (size_t)S * a.stage_bytes;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(zero + a.stage_bytes);
+
+  // ---- per-expert tables and the padding prefix sum (one warp) ----
+  const int E = a.E;
+  for (int e = lane; e <= E; e += 32) s_off[e] = __ldg(a.offsets + e);
+  for (int e = lane; e < E; e += 32) s_cnt[e] = __ldg(a.counts + e);
+  __syncwarp();
+  int bad = 0;
+  int run = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    int pad = 0;
+    if (e < E) {
+      pad = (s_off[e + 1] - s_off[e]) - s_cnt[e];
+      if (pad < 0 || pad >= kTile || s_cnt[e] < 0) {
+        bad = 1;
+        pad = 0;
+      }
+    }
+    const int incl = warp_inclusive_scan(pad);
+    if (e < E) s_padpref[e] = run + incl - pad;
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) s_padpref[E] = run;
+  const int64_t P = s_off[E];
+  if (__any_sync(0xffffffffu, bad) || P > a.P_cap || s_off[0] != 0) {
+    if (lane == 0) record_error(a.status, MOE_ERR_BOUNDS);
+    return;
+  }
+  __syncwarp();
+
+  // ---- this CTA's share of the virtual rows ----
+  const int64_t TK = a.T * a.K;
+  const int64_t V = TK + run;
+  const int64_t G = gridDim.x;
+  const int64_t v0 = V * blockIdx.x / G;
+  const int64_t v1 = V * (blockIdx.x + 1) / G;
+
+  // ---- ring set-up ----
+  for (uint32_t i = lane * 16; i < a.stage_bytes; i += 32 * 16)
+    *reinterpret_cast<uint4*>(zero + i) = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_shared();
+  if (lane == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
+    fence_mbarrier_init();
+  }
+  __syncwarp();
+
+  const int nch = a.n_chunks;
+  const int64_t sl_end = v1 < TK ? v1 : TK;
+  const int64_t t_first = v0 < sl_end ? v0 / a.K : 0;
+  const int64_t n_units = v0 < sl_end ? ((sl_end - 1) / a.K - t_first + 1) * nch : 0;
+
+  auto unit_token = [&](int64_t u) { return t_first + u / nch; };
+  auto issue_load = [&](int64_t u) {  // lane 0 only
+    const int s = (int)(u % S);
+    const int ch = (int)(u % nch);
+    const uint32_t len = chunk_len(a, ch);
+    const uint8_t* src = a.x + unit_token(u) * a.x_stride_bytes + (int64_t)ch * a.chunk_cap;
+    mbar_arrive_expect_tx(&bar[s], len);
+    bulk_load_g2s(stage0 + (size_t)s * a.stage_bytes, src, len, &bar[s]);
+  };
+  // Release +1 for every placed row of token t inside [v0, v1).
+  auto release_token = [&](int64_t t) {  // lane 0 only
+    const int64_t sa = max(v0, t * a.K), sb = min(sl_end, (t + 1) * a.K);
+    for (int64_t sl = sa; sl < sb; ++sl) {
+      const int32_t r = __ldg(a.dst_row + sl);
+      if (r >= 0 && (int64_t)r < a.P_cap) atomic_add_acq_rel_gpu(a.tile_ready + r / kTile, 1u);
+    }
+  };
+
+  int64_t issued = 0;
+  if (lane == 0)
+    for (; issued < n_units && issued < S; ++issued) issue_load(issued);
+
+  int64_t u_fail = -1;
+  for (int64_t u = 0; u < n_units; ++u) {
+    const int s = (int)(u % S);
+    const uint32_t parity = (uint32_t)((u / S) & 1);
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait_bounded(&bar[s], parity) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) {
+      u_fail = u;
+      break;
+    }
+    const int64_t t = unit_token(u);
+    const int ch = (int)(u % nch);
+    const int64_t sa = max(v0, t * a.K), sb = min(sl_end, (t + 1) * a.K);
+
+    if (ch == 0 && a.scale_cols > 0) {  // FP8 scale row, all lanes
+      for (int64_t sl = sa; sl < sb; ++sl) {
+        const int64_t r = checked_row(a, sl);
+        if (r < 0) continue;
+        for (int c = lane; c < a.scale_cols; c += 32)
+          a.xp_scales[r * a.scale_cols + c] = __ldg(a.x_scales + t * a.xs_stride + c);
+      }
+    }
+    if (lane == 0) {
+      const uint32_t len = chunk_len(a, ch);
+      const uint8_t* src = stage0 + (size_t)s * a.stage_bytes;
+      for (int64_t sl = sa; sl < sb; ++sl) {
+        const int64_t r = checked_row(a, sl);
+        if (r < 0) continue;
+        bulk_store_s2g(a.xp + r * a.row_bytes + (int64_t)ch * a.chunk_cap, src, len);
+      }
+      bulk_commit();
+    }
+    if (a.tile_ready) {
+      __syncwarp();  // scale stores of the lanes precede lane 0's release
+      if (lane == 0) {
+        bulk_wait_all<kRelLag>();  // groups <= u - kRelLag have completed
+        fence_proxy_async_global();
+        const int64_t ur = u - kRelLag;
+        if (ur >= 0 && (ur % nch) == nch - 1) release_token(unit_token(ur));
+      }
+    }
+    if (lane == 0) {
+      bulk_wait_read<1>();  // the stores of unit u-1 have read their stage
+      if (u >= 1 && issued < n_units) {
+        issue_load(issued);  // lands in the stage unit u-1 used: (u-1+S) % S
+        ++issued;
+      }
+    }
+  }
+
+  if (u_fail >= 0) {
+    if (lane == 0) {
+      record_error(a.status, MOE_ERR_TIMEOUT);
+      bulk_wait_all<0>();
+      // give the other loads still in flight a bounded chance to land before
+      // the CTA's shared memory is released
+      for (int64_t u = u_fail + 1; u < issued; ++u)
+        if (!mbar_wait_bounded(&bar[u % S], (uint32_t)((u / S) & 1))) break;
+    }
+    return;
+  }
+
+  // ---- padding rows of this range: zero bytes (and zero scales) ----
+  const int64_t q0 = max(v0, TK) - TK, q1 = v1 - TK;
+  if (q1 > q0) {
+    // expert holding padding index q0
+    int e = 0;
+    {
+      int lo = 0, hi = E - 1;  // last e with padpref[e] <= q0
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_padpref[mid] <= q0) lo = mid; else hi = mid - 1;
+      }
+      e = lo;
+    }
+    for (int64_t q = q0; q < q1; ++q) {
+      while (q >= s_padpref[e + 1]) ++e;
+      const int64_t r = (int64_t)s_off[e] + s_cnt[e] + (q - s_padpref[e]);
+      if (a.scale_cols > 0)
+        for (int c = lane; c < a.scale_cols; c += 32) a.xp_scales[r * a.scale_cols + c] = 0.0f;
+      if (lane == 0) {
+        for (int ch = 0; ch < nch; ++ch)
+          bulk_store_s2g(a.xp + r * a.row_bytes + (int64_t)ch * a.chunk_cap, zero,
+                         chunk_len(a, ch));
+        bulk_commit();
+      }
+    }
+  }
+
+  // ---- drain, then release what is still pending ----
+  __syncwarp();
+  if (lane == 0) {
+    bulk_wait_all<0>();
+    if (a.tile_ready) {
+      fence_proxy_async_global();
+      for (int64_t ur = max((int64_t)0, n_units - kRelLag); ur < n_units; ++ur)
+        if ((ur % nch) == nch - 1) release_token(unit_token(ur));
+      if (q1 > q0) {
+        int e = 0;
+        while (e < E - 1 && s_padpref[e + 1] <= q0) ++e;
+        int64_t q = q0;
+        while (q < q1) {
+          while (q >= s_padpref[e + 1]) ++e;
+          const int64_t q_end = min(q1, (int64_t)s_padpref[e + 1]);
+          const int64_t last_row = (int64_t)s_off[e] + s_cnt[e] + (q_end - 1 - s_padpref[e]);
+          atomic_add_acq_rel_gpu(a.tile_ready + last_row / kTile, (uint32_t)(q_end - q));
+          q = q_end;
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
+                                    int64_t x_row_stride, const float* x_scales,
+                                    int64_t x_scales_row_stride, const int32_t* dst_row, int K,
+                                    const int32_t* expert_counts, const int32_t* expert_offsets,
+                                    int E, void* xp, float* xp_scales, int64_t P_cap,
+                                    uint32_t* tile_ready, int32_t* d_status, void* stream) {
+  using namespace moe;
+  if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (T < 0 || H <= 0 || K < 1 || K > MOE_MAX_TOPK || E < 1 || E > MOE_MAX_EXPERTS)
+    return MOE_ERR_INVALID_ARG;
+  if (T * (int64_t)K > (int64_t)INT32_MAX || P_cap > (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (P_cap < moe_padded_capacity(T, K, E)) return MOE_ERR_CAPACITY;
+  if (x_row_stride < H) return MOE_ERR_INVALID_ARG;
+  const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 1;
+  const int64_t row_bytes = (int64_t)H * elem;
+  if (row_bytes % 16 != 0 || (x_row_stride * elem) % 16 != 0) return MOE_ERR_INVALID_ARG;
+  if (!xp || !expert_counts || !expert_offsets || (T > 0 && (!x || !dst_row)))
+    return MOE_ERR_INVALID_ARG;
+  if (!moe_host::aligned16(xp) || (x && !moe_host::aligned16(x))) return MOE_ERR_INVALID_ARG;
+  int scale_cols = 0;
+  if (dtype == MOE_DTYPE_E4M3) {
+    if (H % 128 != 0 || !xp_scales || (T > 0 && !x_scales)) return MOE_ERR_INVALID_ARG;
+    scale_cols = H / 128;
+    if (x_scales_row_stride < scale_cols) return MOE_ERR_INVALID_ARG;
+  } else if (x_scales || xp_scales) {
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (T == 0) return MOE_OK;  // P = 0: nothing to write
+
+  PermArgs a;
+  a.x = static_cast<const uint8_t*>(x);
+  a.x_stride_bytes = x_row_stride * elem;
+  a.row_bytes = row_bytes;
+  a.x_scales = x_scales;
+  a.xs_stride = x_scales_row_stride;
+  a.scale_cols = scale_cols;
+  a.dst_row = dst_row;
+  a.T = T;
+  a.K = K;
+  a.counts = expert_counts;
+  a.offsets = expert_offsets;
+  a.E = E;
+  a.xp = static_cast<uint8_t*>(xp);
+  a.xp_scales = xp_scales;
+  a.P_cap = P_cap;
+  a.tile_ready = tile_ready;
+  a.status = d_status;
+  a.chunk_cap = (uint32_t)(row_bytes < (int64_t)kMaxChunk ? row_bytes : kMaxChunk);
+  a.stage_bytes = (a.chunk_cap + 127u) / 128u * 128u;
+  a.n_chunks = (int)((row_bytes + a.chunk_cap - 1) / a.chunk_cap);
+
+  const int dev = moe_host::current_device();
+  int optin = 0;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const size_t static_smem = (3 * MOE_MAX_EXPERTS + 2) * sizeof(int32_t);
+  const size_t per_cta = (size_t)optin / kPermCtasPerSm - static_smem - 1024;
+  int stages = (int)((per_cta - a.stage_bytes - kMaxStages * 8) / a.stage_bytes);
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 2) stages = 2;
+  a.stages = stages;
+  const size_t dyn = (size_t)(stages + 1) * a.stage_bytes + (size_t)stages * 8;
+  if (dyn + static_smem > (size_t)optin) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)dyn) != cudaSuccess)
+    return MOE_ERR_CUDA;
+
+  const int64_t v_bound = T * K + (int64_t)(kTile - 1) * E;
+  int64_t grid = (int64_t)moe_host::sm_count(dev) * kPermCtasPerSm;
+  const int64_t by_work = (v_bound + 7) / 8;
+  if (grid > by_work) grid = by_work;
+  if (grid < 1) grid = 1;
+  permute_kernel<<<(unsigned)grid, 32, dyn, static_cast<cudaStream_t>(stream)>>>(a);
+  return moe_host::launch_status();
+}

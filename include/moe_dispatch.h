@@ -1,0 +1,242 @@
+/*
+ * moe_dispatch.h -- C ABI of the single-GPU MoE token dispatch / combine
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * The operations and where they are defined:
+ *   [ASC]   Huawei torch_npu "npu_moe_distribute_combine" API reference:
+ *           function description (combine = the dispatch path walked back,
+ *           expert outputs multiplied by their weights and summed, plus the
+ *           shared expert) and the parameters expert_ids, expand_x,
+ *           expand_idx, ep_send_counts, expert_scales, shared_expert_x,
+ *           moe_expert_num, H, BS, K.
+ *   [DEP]   DeepEP pull request "Intra-node compute compensation + overlap
+ *           robustness (CUDA719 fix)", section "Kernel / host": the fused
+ *           unzip that scatters token rows and the mapping table into expert
+ *           buffers, its chunk-completion counter updated with
+ *           atom.acq_rel.gpu, one acquire per chunk on the consumer side, and
+ *           bounds guards on every write.
+ *   [TEMPO] TEMPO summary (makespan-aware expert load balancing), section 1:
+ *           grouped GEMMs round each expert's tokens up to 128-token M-tiles.
+ *
+ * Notation: T tokens, H hidden size, E routed experts, K experts per token,
+ * R logical expert-parallel ranks (expert e belongs to rank e / (E/R)),
+ * c_e = number of (t, k) slots routed to expert e, offsets are exclusive
+ * prefix sums of 128 * ceil(c_e / 128), P = offsets[E] <= P_cap.
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers unless stated; the caller owns every
+ *     buffer; the library allocates no memory and keeps no state besides
+ *     per-device launch settings.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     enqueued on it; no call synchronises the host.
+ *   - bf16 = IEEE bfloat16 (2 bytes), E4M3 = OCP 8-bit float E4M3 (1 byte).
+ *   - Row-major layouts; "[A, B]" = A rows of B elements.
+ *   - Return value: MOE_OK if the work was enqueued.  Argument errors that
+ *     the host can see (NULL where not allowed, sizes out of range, bad
+ *     alignment, E % R != 0, capacity too small) return at once and launch
+ *     nothing.  MOE_ERR_CUDA if a launch failed.
+ *   - `d_status`: device int32, set to 0 by the caller before a sequence of
+ *     calls.  Errors that depend on data (an expert id out of range, a
+ *     repeated id, a row index outside the buffers, a timed-out wait) are
+ *     written there with first-writer-wins semantics; the kernel then skips
+ *     the offending writes instead of trapping.  Read it after the stream
+ *     has been synchronised.  Outputs are unspecified (but every write stays
+ *     inside the buffers) when it is non-zero.
+ */
+#ifndef MOE_DISPATCH_H_
+#define MOE_DISPATCH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_TILE_M 128 /* rows per M-tile ([TEMPO] section 1) */
+#define MOE_MAX_EXPERTS 512 /* [ASC] moe_expert_num in [1, 512] */
+#define MOE_MAX_TOPK 16     /* [ASC] K <= 16 */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,      /* host-side argument check failed */
+  MOE_ERR_EXPERT_RANGE = 2,     /* an expert id outside [0, E) */
+  MOE_ERR_DUPLICATE_EXPERT = 3, /* an expert id repeated within a token's row */
+  MOE_ERR_CAPACITY = 4,         /* P_cap below moe_padded_capacity(T, K, E) */
+  MOE_ERR_TIMEOUT = 5,          /* a bounded device-side wait gave up */
+  MOE_ERR_CUDA = 6,             /* a CUDA launch or attribute call failed */
+  MOE_ERR_UNSUPPORTED = 7,      /* dtype or device not supported */
+  MOE_ERR_BOUNDS = 8            /* a row index pointed outside its buffer */
+} moe_status_t;
+
+typedef enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_E4M3 = 1 } moe_dtype_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+MOE_API const char* moe_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+MOE_API int moe_version(void);
+
+/*
+ * Upper bound on the padded row count P for T tokens, K slots per token and
+ * E experts, rounded up to a multiple of 128:  T*K + 127*min(E, T*K).
+ * Every expert-major buffer (xp, y, grad_y) needs at least this many rows.
+ * Returns -1 if an argument is out of range.
+ */
+MOE_API int64_t moe_padded_capacity(int64_t T, int K, int E);
+
+/* Bytes of device scratch that moe_dispatch_layout needs (256-byte aligned
+ * start).  0 is never returned for valid sizes; -1 cast to size_t on bad
+ * arguments. */
+MOE_API size_t moe_layout_workspace_bytes(int64_t T, int K, int E);
+
+/*
+ * Dispatch layout.  [ASC] expert_ids (validation), expand_idx and
+ * ep_send_counts (counts in prefix-sum form); [TEMPO] 128-row padding;
+ * [DEP] the mapping table written by the fused unzip.
+ *
+ * In:
+ *   topk_idx      int32 [T, K], contiguous; ids in [0, E), distinct per row.
+ *   T >= 0, 1 <= K <= 16, 1 <= E <= 512, 1 <= R <= E with E % R == 0,
+ *   T*K <= 2^31 - 1, P_cap >= moe_padded_capacity(T, K, E), P_cap < 2^31.
+ * Out:
+ *   expert_counts  int32 [E]     c_e
+ *   expert_offsets int32 [E+1]   exclusive prefix sum of 128*ceil(c_e/128);
+ *                                expert_offsets[E] = P
+ *   rank_counts    int32 [R]     sum of c_e over the experts of rank r
+ *   rank_offsets   int32 [R+1]   expert_offsets[r*E/R]; rank_offsets[R] = P
+ *   dst_row        int32 [T*K]   row of slot (t,k) in the expert-major
+ *                                buffer: expert_offsets[e] + number of
+ *                                earlier tokens routed to e (stable, token
+ *                                order); -1 for an out-of-range id
+ *   row_src        int32 [P_cap] (nullable) slot t*K+k stored in each row,
+ *                                -1 for padding rows and rows >= P
+ *   tile_ready     uint32 [ceil(P_cap/128)] (nullable) chunk-completion
+ *                                counters, all set to 0 here
+ * Scratch: workspace of workspace_bytes >= moe_layout_workspace_bytes(),
+ *   256-byte aligned; its contents need no initialisation.
+ * Data errors: MOE_ERR_EXPERT_RANGE (that slot is not placed),
+ *   MOE_ERR_DUPLICATE_EXPERT (both slots are still placed).
+ * Results are bit-exact and independent of launch configuration.
+ */
+MOE_API int moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int K, int E, int R,
+                        int32_t* expert_counts, int32_t* expert_offsets,
+                        int32_t* rank_counts, int32_t* rank_offsets, int32_t* dst_row,
+                        int32_t* row_src, uint32_t* tile_ready, int64_t P_cap,
+                        int32_t* d_status, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
+ * Dispatch permute (the fused unzip of [DEP]; produces [ASC] expand_x).
+ *   xp[dst_row[t*K+k]] = x[t]  for every placed slot, byte for byte;
+ *   padding rows [offsets[e] + counts[e], offsets[e+1]) = 0 (E4M3: code
+ *   0x00 and scale 0.0f); rows >= P untouched.
+ *
+ * In:
+ *   x        [T, H] of `dtype`, row stride x_row_stride elements (>= H);
+ *            16-byte aligned base, row bytes and stride multiples of 16
+ *            (bf16: H % 8 == 0; E4M3: H % 128 == 0).
+ *   x_scales fp32 [T, H/128], row stride x_scales_row_stride (E4M3 only;
+ *            NULL for bf16).
+ *   dst_row, expert_counts, expert_offsets: as produced by the layout call.
+ * Out:
+ *   xp        [P_cap, H] of `dtype`, contiguous, 16-byte aligned.
+ *   xp_scales fp32 [P_cap, H/128] (E4M3 only; NULL for bf16).
+ *   tile_ready (nullable) counters zeroed by the layout call; each finished
+ *            row adds 1 to tile_ready[row/128] with atom.add.acq_rel.gpu
+ *            after its bytes (and scales) are globally visible, so a tile
+ *            whose counter reads 128 with an acquire load is complete.
+ * Data errors: MOE_ERR_BOUNDS if a dst_row entry or offset leaves
+ *   [0, P_cap) (that write is skipped); MOE_ERR_TIMEOUT if a staged load
+ *   did not land within about 2 s.
+ */
+MOE_API int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H, int64_t x_row_stride,
+                         const float* x_scales, int64_t x_scales_row_stride,
+                         const int32_t* dst_row, int K, const int32_t* expert_counts,
+                         const int32_t* expert_offsets, int E, void* xp, float* xp_scales,
+                         int64_t P_cap, uint32_t* tile_ready, int32_t* d_status,
+                         void* stream);
+
+/*
+ * Combine ([ASC] function description, expert_scales, shared_expert_x):
+ *   out[t] = bf16( sum_{k=0..K-1} scales[t,k] * y[dst_row[t*K+k]] + shared_x[t] )
+ * computed per element in fp32: acc = 0; acc = fma(scales[t,k], y, acc) for
+ * k = 0, 1, ..., K-1 in that order; acc = acc + shared_x; one round-to-
+ * nearest-even to bf16.  The shared-expert term has no weight.
+ *
+ * In:  y bf16 [P_cap, H] contiguous; scales fp32 [T, K]; dst_row int32 [T*K];
+ *      shared_x bf16 [T, H] or NULL (no shared expert).
+ * Out: out bf16 [T, H] contiguous.
+ * H % 8 == 0; y, shared_x, out 16-byte aligned.
+ * Slots with dst_row == -1 add nothing; other out-of-range rows set
+ * MOE_ERR_BOUNDS and add nothing.
+ */
+MOE_API int moe_combine(const void* y, const int32_t* dst_row, const float* scales,
+                const void* shared_x, int64_t T, int K, int H, int64_t P_cap, void* out,
+                int32_t* d_status, void* stream);
+
+/*
+ * Backward of combine (out is linear in y and in scales):
+ *   grad_y[dst_row[t*K+k]] = bf16( scales[t,k] * grad_out[t] )   (fp32 product)
+ *   grad_scales[t*K+k]     = sum_h grad_out[t,h] * y[dst_row[t*K+k], h]
+ *                            (fp32, fixed order for a given H)
+ *   padding rows of grad_y below P are set to 0; rows >= P untouched.
+ * In:  grad_out bf16 [T, H]; y bf16 [P_cap, H]; scales fp32 [T, K];
+ *      dst_row, expert_counts, expert_offsets from the layout call.
+ * Out: grad_y bf16 [P_cap, H]; grad_scales fp32 [T, K].
+ */
+MOE_API int moe_combine_bwd(const void* grad_out, const void* y, const float* scales,
+                    const int32_t* dst_row, const int32_t* expert_counts,
+                    const int32_t* expert_offsets, int E, int64_t T, int K, int H,
+                    int64_t P_cap, void* grad_y, float* grad_scales, int32_t* d_status,
+                    void* stream);
+
+/*
+ * Backward of dispatch (the permute copies x[t] into K rows; its adjoint
+ * adds them back):
+ *   grad_x[t] = bf16( sum_{k in order} grad_xp[dst_row[t*K+k]] )   (fp32 adds)
+ * In:  grad_xp bf16 [P_cap, H]; dst_row int32 [T*K].   Out: grad_x bf16 [T, H].
+ */
+MOE_API int moe_dispatch_bwd(const void* grad_xp, const int32_t* dst_row, int64_t T, int K, int H,
+                     int64_t P_cap, void* grad_x, int32_t* d_status, void* stream);
+
+/*
+ * E4M3 quantisation with one fp32 scale per 128 channels (the FP8 dispatch
+ * input: codes plus scales carried alongside).  Per token t and block b:
+ *   s = amax|x| / 448 in fp32 (1 if amax == 0);
+ *   q = E4M3(x / s) with fp32 division, round-to-nearest-even, saturating
+ *       at +-448.
+ * In:  x bf16 [T, H], row stride x_row_stride elements; H % 128 == 0.
+ * Out: q uint8 [T, H] contiguous; q_scales fp32 [T, H/128] contiguous.
+ */
+MOE_API int moe_quantize_e4m3(const void* x, int64_t T, int H, int64_t x_row_stride, void* q,
+                      float* q_scales, int32_t* d_status, void* stream);
+
+/*
+ * Reference consumer of the chunk-completion counters ([DEP]: one acquire
+ * per chunk).  For every tile j < P/128 (P = expert_offsets[E]) it polls
+ * tile_ready[j] with ld.acquire.gpu until it reads 128, at most timeout_ns
+ * nanoseconds, then reads the tile and writes
+ *   checksums[j] = sum_i w_i * (2i + 1)  mod 2^32
+ * over the tile's 32-bit words w_i (128 rows of row_bytes, then, when
+ * xp_scales is given, 128 scale rows of 4*scale_cols bytes).  A wait that
+ * runs out sets MOE_ERR_TIMEOUT and leaves checksums[j] unwritten; once the
+ * status is non-zero no further wait is started.
+ * row_bytes % 4 == 0; checksums uint32 [ceil(P_cap/128)].
+ */
+MOE_API int moe_wait_tiles_checksum(const uint32_t* tile_ready, const int32_t* expert_offsets, int E,
+                            const void* xp, int64_t row_bytes, const float* xp_scales,
+                            int scale_cols, int64_t P_cap, uint32_t* checksums,
+                            int64_t timeout_ns, int32_t* d_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_DISPATCH_H_ */

@@ -1,0 +1,175 @@
+"""GPU parity: combine, combine backward and dispatch backward against the CPU
+oracle, on the workloads' sizes and on ragged edge shapes.
+
+Tolerance (bf16 outputs): the oracle rounds the exact sum once; the kernel
+rounds an fp32 running sum, so |gpu - ref| <= 2^-7 |ref| + gamma_n * sum|terms|
+(see _gpu_util.assert_bf16_close).  In practice nearly every element is
+bit-identical, which the tests also report.  grad_scales is an fp32 dot
+product over H terms in a fixed but different order than the oracle's double
+sum: |err| <= gamma_H * sum_h |g_h y_h| + 2^-24 |ref|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _gpu_util import assert_bf16_close, dev_u16, ensure_lib, f64, gamma
+from combine_moe_dispatch_05_b200 import ops
+from combine_moe_dispatch_05_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    ensure_lib()
+
+
+def prepare(s, identity=False):
+    ids = W.topk_ids(s)
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    st = ops.new_status()
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R, status=st)
+    assert ops.read_status(st) == 0
+    scales = W.topk_scales(s)
+    if identity:  # y = the dispatched x (identity experts)
+        x = W.tokens(s)
+        y = np.zeros((ref.P_cap, s.H), np.uint16)
+        oracle.permute_rows(W.as_u16(x), ref.dst_row, s.K, ref.counts, ref.offsets, y)
+        y_cpu = W.from_u16(y)
+    else:
+        y_cpu = W.expert_out(s, ref.P_cap)
+    return L, ref, scales, y_cpu
+
+
+def combine_mag(y_u16, dst_row, scales, shared_u16=None):
+    T, K = scales.shape
+    g = np.abs(f64(y_u16)[dst_row.reshape(T, K)])           # [T, K, H]
+    m = np.einsum("tk,tkh->th", np.abs(scales.astype(np.float64)), g)
+    if shared_u16 is not None:
+        m = m + np.abs(f64(shared_u16))
+    return m
+
+
+def check_combine(s, shared=False, identity=False):
+    L, ref, scales, y_cpu = prepare(s, identity)
+    sh_cpu = W.shared_out(s) if shared else None
+    st = ops.new_status()
+    out = ops.moe_combine(y_cpu.to(DEV), L.dst_row, scales.to(DEV),
+                          shared_x=None if sh_cpu is None else sh_cpu.to(DEV), status=st)
+    assert ops.read_status(st) == 0
+    y = W.as_u16(y_cpu)
+    sh = None if sh_cpu is None else W.as_u16(sh_cpu)
+    out_ref = oracle.combine(y, ref.dst_row, scales.numpy(), sh)
+    mag = combine_mag(y, ref.dst_row, scales.numpy(), sh)
+    exact = assert_bf16_close(dev_u16(out), out_ref, mag, s.K + 1, "combine")
+    assert exact > 0.99, exact
+    return out, out_ref
+
+
+@pytest.mark.parametrize("cfg,shared,identity", [(1, False, True), (1, False, False),
+                                                 (2, False, False), (4, True, False)])
+def test_combine_parity_workloads(cfg, shared, identity):
+    check_combine(W.config(cfg), shared, identity)
+
+
+def test_combine_identity_experts_returns_x_within_an_ulp():
+    """Tiny workload, identity experts: out = x * sum_k s_k with sum_k s_k = 1
+    up to fp32 rounding, so out equals x to within one bf16 ulp."""
+    s = W.config(1)
+    out, _ = check_combine(s, identity=True)
+    x = f64(W.as_u16(W.tokens(s)))
+    assert np.all(np.abs(f64(dev_u16(out)) - x) <= 2.0 ** -7 * np.abs(x) + 1e-30)
+
+
+@pytest.mark.parametrize("T,H,E,K,R,shared", [
+    (1, 8, 1, 1, 1, False), (3, 16, 4, 2, 2, True), (129, 24, 9, 3, 3, False),
+    (513, 520, 33, 5, 1, True), (40, 7176, 17, 16, 1, False), (1000, 64, 512, 16, 8, True)])
+def test_combine_parity_edge_shapes(T, H, E, K, R, shared):
+    check_combine(W.Spec("edge", T, H, E, K, R, "uniform", seed=3 + T * H), shared)
+
+
+def test_combine_one_hot_is_bit_exact():
+    s = W.config(4)
+    L, ref, scales, y_cpu = prepare(s)
+    oh = torch.zeros_like(scales)
+    oh[:, 3] = 1.0
+    out = ops.moe_combine(y_cpu.to(DEV), L.dst_row, oh.to(DEV))
+    rows = ref.dst_row.reshape(s.T, s.K)[:, 3]
+    assert np.array_equal(dev_u16(out), W.as_u16(y_cpu)[rows])
+
+
+# ------------------------------------------------------------ backward ----
+def check_combine_bwd(s):
+    L, ref, scales, y_cpu = prepare(s)
+    g_cpu = W.grad_out(s)
+    SENT = 0x3C3C
+    gy = torch.full((L.P_cap, s.H), 0, dtype=torch.bfloat16, device=DEV)
+    gy.view(torch.int16).fill_(SENT)
+    st = ops.new_status()
+    gy, gs = ops.moe_combine_bwd(g_cpu.to(DEV), y_cpu.to(DEV), scales.to(DEV), L, grad_y=gy,
+                                 status=st)
+    assert ops.read_status(st) == 0
+    g, y = W.as_u16(g_cpu), W.as_u16(y_cpu)
+    gy_ref = np.full((ref.P_cap, s.H), SENT, np.uint16)
+    gs_ref = oracle.combine_bwd(g, y, scales.numpy(), ref.dst_row, ref.counts, ref.offsets, gy_ref)
+    got = dev_u16(gy)
+    # rows that hold a slot: one product rounded twice (fp32 then bf16) vs once
+    real = ref.row_src >= 0
+    mag = np.abs(f64(gy_ref[real]))
+    assert_bf16_close(got[real], gy_ref[real], mag, 1, "grad_y")
+    assert np.array_equal(got[~real], gy_ref[~real])          # zero padding, untouched tail
+    T, K = s.T, s.K
+    rows = ref.dst_row.reshape(T, K)
+    dmag = np.einsum("th,tkh->tk", np.abs(f64(g)), np.abs(f64(y)[rows]))
+    err = np.abs(gs.cpu().numpy().astype(np.float64) - gs_ref.astype(np.float64))
+    assert np.all(err <= gamma(s.H) * dmag + 2.0 ** -24 * np.abs(gs_ref) + 1e-30)
+
+
+def check_dispatch_bwd(s):
+    L, ref, _, y_cpu = prepare(s)
+    st = ops.new_status()
+    gx = ops.moe_dispatch_bwd(y_cpu.to(DEV), L.dst_row, s.T, s.K, status=st)
+    assert ops.read_status(st) == 0
+    y = W.as_u16(y_cpu)
+    ref_out = oracle.dispatch_bwd(y, ref.dst_row, s.T, s.K)
+    ones = np.ones((s.T, s.K), np.float32)
+    mag = combine_mag(y, ref.dst_row, ones)
+    exact = assert_bf16_close(dev_u16(gx), ref_out, mag, s.K, "dispatch_bwd")
+    assert exact > 0.99
+
+
+@pytest.mark.parametrize("variant", ["p60", "p100"])
+def test_backward_parity_skewed_workload(variant):
+    s = W.config(5)
+    if variant == "p100":
+        s = s.with_(hot_p=1.0)
+    check_combine_bwd(s)
+    check_dispatch_bwd(s)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 4])
+def test_backward_parity_workloads(cfg):
+    s = W.config(cfg)
+    check_combine_bwd(s)
+    check_dispatch_bwd(s)
+
+
+@pytest.mark.parametrize("T,H,E,K,R", [(1, 8, 1, 1, 1), (77, 24, 6, 3, 2), (300, 1032, 40, 16, 4),
+                                       (2, 7168, 256, 8, 8)])
+def test_backward_parity_edge_shapes(T, H, E, K, R):
+    s = W.Spec("edge", T, H, E, K, R, "uniform", seed=11 + T + H)
+    check_combine_bwd(s)
+    check_dispatch_bwd(s)
+
+
+@pytest.mark.parametrize("K", [2, 4, 8])
+def test_dispatch_bwd_of_dispatch_is_exactly_K_x(K):
+    s = W.Spec("k", 600, 264, 24, K, 4, "uniform", seed=900 + K)
+    ids = W.topk_ids(s)
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R)
+    x = W.tokens(s).to(DEV)
+    xp = ops.moe_dispatch_permute(x, L)
+    gx = ops.moe_dispatch_bwd(xp, L.dst_row, s.T, s.K)
+    assert torch.equal(gx.float(), x.float() * K)

@@ -1,0 +1,141 @@
+"""GPU: chunk-completion counters and the reference consumer.
+
+A consumer that acquires a tile's counter at 128 must see the whole tile
+(content checksums equal the oracle's); a consumer with no producer must give
+up within its time limit and report MOE_ERR_TIMEOUT, leaving the context
+usable.  Device-side data errors are reported through the status word and
+the offending writes are skipped.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _gpu_util import assert_bf16_close, dev_u16, ensure_lib, f64
+from combine_moe_dispatch_05_b200 import ops
+from combine_moe_dispatch_05_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    ensure_lib()
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 4])
+def test_consumer_sees_complete_tiles_bf16(cfg):
+    s = W.config(cfg)
+    ids = W.topk_ids(s)
+    x = W.tokens(s)
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    xp_ref = np.zeros((ref.P_cap, s.H), np.uint16)
+    oracle.permute_rows(W.as_u16(x), ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    cs_ref = oracle.tile_checksums(xp_ref, ref.P // 128)
+
+    st = ops.new_status()
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R, status=st)
+    xp = ops.moe_dispatch_permute(x.to(DEV), L, status=st)
+    cs = ops.moe_wait_tiles_checksum(L, xp, status=st, timeout_ns=2 * 10**9)
+    assert ops.read_status(st) == 0
+    got = cs.cpu().numpy().view(np.uint32)[:ref.P // 128]
+    assert np.array_equal(got, cs_ref)
+
+
+def test_consumer_sees_complete_tiles_fp8_with_scales():
+    s = W.config(3).with_(T=3000, H=1024, E=32, K=4, R=4)
+    ids = W.topk_ids(s)
+    codes, xs = W.e4m3_codes(s), W.block_scales(s)
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    xp_ref = np.zeros((ref.P_cap, s.H), np.uint8)
+    xps_ref = np.zeros((ref.P_cap, s.H // 128), np.float32)
+    oracle.permute_rows(codes.numpy(), ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    oracle.permute_rows(xs.numpy(), ref.dst_row, s.K, ref.counts, ref.offsets, xps_ref)
+    cs_ref = oracle.tile_checksums(xp_ref, ref.P // 128, xps_ref)
+    st = ops.new_status()
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R, status=st)
+    xp, xps = ops.moe_dispatch_permute(codes.to(DEV), L, x_scales=xs.to(DEV), status=st)
+    cs = ops.moe_wait_tiles_checksum(L, xp, xps, status=st)
+    assert ops.read_status(st) == 0
+    assert np.array_equal(cs.cpu().numpy().view(np.uint32)[:ref.P // 128], cs_ref)
+
+
+def test_consumer_without_producer_times_out_and_context_survives():
+    s = W.config(1)
+    ids = W.topk_ids(s)
+    st = ops.new_status()
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R, status=st)   # counters reset to 0
+    xp = torch.zeros((L.P_cap, s.H), dtype=torch.bfloat16, device=DEV)
+    assert ops.read_status(st) == 0
+    ops.moe_wait_tiles_checksum(L, xp, status=st, timeout_ns=20 * 10**6)   # 20 ms
+    assert ops.read_status(st) == ops.ERR_TIMEOUT
+    # the context is still usable: a normal dispatch succeeds afterwards
+    st2 = ops.new_status()
+    xp2 = ops.moe_dispatch_permute(W.tokens(s).to(DEV), L, status=st2)
+    cs = ops.moe_wait_tiles_checksum(L, xp2, status=st2)
+    assert ops.read_status(st2) == 0
+
+
+def test_permute_without_counters_leaves_them_alone():
+    s = W.config(1)
+    ids = W.topk_ids(s)
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R)
+    ops.moe_dispatch_permute(W.tokens(s).to(DEV), L, use_counters=False)
+    assert int(L.tile_ready.abs().sum()) == 0
+
+
+def test_bounds_guard_skips_rows_outside_the_buffer():
+    """A corrupted dst_row entry (host-made fault) is reported and its write is
+    skipped; guard rows around the buffer stay intact."""
+    s = W.config(1)
+    ids = W.topk_ids(s)
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R)
+    torch.cuda.synchronize()
+    L.dst_row[7] = L.P_cap + 5          # outside [0, P_cap)
+    L.dst_row[9] = -12
+    guard = torch.full((L.P_cap + 64, s.H), 0, dtype=torch.bfloat16, device=DEV)
+    guard.view(torch.int16).fill_(0x1234)
+    xp = guard[:L.P_cap]
+    st = ops.new_status()
+    ops.moe_dispatch_permute(W.tokens(s).to(DEV), L, xp=xp, status=st)
+    assert ops.read_status(st) == ops.ERR_BOUNDS
+    assert bool((guard[L.P_cap:].view(torch.int16) == 0x1234).all())
+    st = ops.new_status()
+    y = torch.zeros((L.P_cap, s.H), dtype=torch.bfloat16, device=DEV)
+    ops.moe_combine(y, L.dst_row, W.topk_scales(s).to(DEV), status=st)
+    assert ops.read_status(st) == ops.ERR_BOUNDS
+    st = ops.new_status()
+    ops.moe_dispatch_bwd(y, L.dst_row, s.T, s.K, status=st)
+    assert ops.read_status(st) == ops.ERR_BOUNDS
+    st = ops.new_status()
+    gy = guard[:L.P_cap]
+    ops.moe_combine_bwd(W.grad_out(s).to(DEV), y, W.topk_scales(s).to(DEV), L, grad_y=gy,
+                        status=st)
+    assert ops.read_status(st) == ops.ERR_BOUNDS
+    assert bool((guard[L.P_cap:].view(torch.int16) == 0x1234).all())
+
+
+def test_out_of_range_ids_are_skipped_downstream():
+    s = W.config(4)
+    ids = W.topk_ids(s)
+    ids[10, 1] = s.E + 3
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    st = ops.new_status()
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R, status=st)
+    assert ops.read_status(st) == ops.ERR_EXPERT_RANGE
+    x = W.tokens(s)
+    st2 = ops.new_status()
+    xp = ops.moe_dispatch_permute(x.to(DEV), L, status=st2)
+    assert ops.read_status(st2) == 0          # -1 rows are skipped silently
+    xp_ref = np.zeros((ref.P_cap, s.H), np.uint16)
+    oracle.permute_rows(W.as_u16(x), ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    assert np.array_equal(dev_u16(xp)[:ref.P], xp_ref[:ref.P])
+    sc = W.topk_scales(s)
+    out = ops.moe_combine(xp, L.dst_row, sc.to(DEV), status=st2)
+    assert ops.read_status(st2) == 0
+    out_ref = oracle.combine(xp_ref, ref.dst_row, sc.numpy(), None)
+    rows = np.where(ref.dst_row >= 0, ref.dst_row, ref.P_cap - 1).reshape(s.T, s.K)
+    mag = np.einsum("tk,tkh->th", np.abs(sc.numpy().astype(np.float64)),
+                    np.abs(f64(xp_ref)[rows]) * (ref.dst_row.reshape(s.T, s.K, 1) >= 0))
+    assert_bf16_close(dev_u16(out), out_ref, mag, s.K + 1, "combine with an unplaced slot")

@@ -1,0 +1,222 @@
+"""GPU parity: dispatch layout and permute against the CPU oracle.
+
+Integer outputs (counts, offsets, rank sums, dst_row, row_src) and permuted
+bytes must match bit for bit; padding rows are zero, rows past P keep their
+previous contents, and every counter of a finished tile reads 128.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _gpu_util import ensure_lib, dev_u16
+from combine_moe_dispatch_05_b200 import ops
+from combine_moe_dispatch_05_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    ensure_lib()
+
+
+def run_layout(ids_cpu: torch.Tensor, E: int, R: int):
+    ids = ids_cpu.to(DEV)
+    st = ops.new_status()
+    L = ops.moe_dispatch_layout(ids, E, R, status=st)
+    return L, ops.read_status(st)
+
+
+def check_layout(ids_cpu, E, R, expect_status=0):
+    T, K = ids_cpu.shape
+    L, st = run_layout(ids_cpu, E, R)
+    ref = oracle.layout(ids_cpu.numpy(), E, R)
+    assert st == ref.status == expect_status
+    assert L.P_cap == ref.P_cap
+    assert np.array_equal(L.expert_counts.cpu().numpy(), ref.counts)
+    assert np.array_equal(L.expert_offsets.cpu().numpy(), ref.offsets)
+    assert np.array_equal(L.rank_counts.cpu().numpy(), ref.rank_counts)
+    assert np.array_equal(L.rank_offsets.cpu().numpy(), ref.rank_offsets)
+    if T:
+        assert np.array_equal(L.dst_row.cpu().numpy()[:T * K], ref.dst_row)
+    assert np.array_equal(L.row_src.cpu().numpy()[:ref.P_cap], ref.row_src)
+    n_tiles = (ref.P_cap + 127) // 128
+    assert np.all(L.tile_ready.cpu().numpy()[:n_tiles] == 0)
+    return L, ref
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("seed_offset", [0, 1])
+def test_layout_parity_workloads(cfg, seed_offset):
+    s = W.config(cfg, seed_offset)
+    check_layout(W.topk_ids(s), s.E, s.R)
+
+
+def test_layout_parity_hot_expert_everywhere():
+    s = W.config(5).with_(hot_p=1.0)
+    check_layout(W.topk_ids(s), s.E, s.R)
+
+
+@pytest.mark.parametrize("T,K,E,R", [
+    (1, 1, 1, 1), (0, 4, 8, 2), (1, 16, 16, 4), (63, 3, 5, 5), (65, 8, 512, 8),
+    (1000, 16, 512, 512), (3000, 1, 2, 2), (129, 2, 3, 1), (257, 7, 64, 16), (4097, 6, 64, 16)])
+def test_layout_parity_edge_shapes(T, K, E, R):
+    s = W.Spec("edge", T, 8, E, K, R, "uniform", seed=77 + T + K + E)
+    ids = W.topk_ids(s) if T else torch.zeros((0, K), dtype=torch.int32)
+    check_layout(ids, E, R)
+
+
+def test_layout_all_tokens_one_expert_multi_tile():
+    ids = torch.full((1000, 1), 3, dtype=torch.int32)
+    L, ref = check_layout(ids, 4, 2)
+    assert ref.offsets.tolist() == [0, 0, 0, 0, 1024]
+
+
+def test_layout_reports_out_of_range_and_duplicates():
+    s = W.config(4)
+    ids = W.topk_ids(s)
+    bad = ids.clone()
+    bad[100, 2] = s.E            # out of range
+    bad[2000, 0] = -3
+    check_layout(bad, s.E, s.R, expect_status=oracle.ERR_EXPERT_RANGE)
+    dup = ids.clone()
+    dup[555, 1] = dup[555, 0]
+    check_layout(dup, s.E, s.R, expect_status=oracle.ERR_DUPLICATE_EXPERT)
+
+
+# ------------------------------------------------------------ permute ----
+SENT = 0x5A
+
+
+def run_permute_bf16(s, x_cpu, strided=False):
+    ids = W.topk_ids(s)
+    L, _ = run_layout(ids, s.E, s.R)
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    if strided:  # rows of a wider buffer
+        wide = torch.zeros((s.T, s.H + 24), dtype=torch.bfloat16)
+        wide[:, 8:8 + s.H] = x_cpu
+        xd = wide.to(DEV)[:, 8:8 + s.H]
+    else:
+        xd = x_cpu.to(DEV)
+    xp = torch.full((L.P_cap, s.H), 0, dtype=torch.bfloat16, device=DEV)
+    xp.view(torch.uint8).fill_(SENT)
+    st = ops.new_status()
+    ops.moe_dispatch_permute(xd, L, xp=xp, status=st)
+    assert ops.read_status(st) == 0
+    xp_ref = np.full((ref.P_cap, s.H), SENT * 0x0101, np.uint16)
+    oracle.permute_rows(W.as_u16(x_cpu), ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    return L, ref, xp, xp_ref
+
+
+def check_counters(L, ref):
+    cnt = L.tile_ready.cpu().numpy().view(np.uint32)
+    n_full = ref.P // 128
+    assert np.all(cnt[:n_full] == 128)
+    assert np.all(cnt[n_full:] == 0)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 4])
+def test_permute_bf16_parity(cfg):
+    s = W.config(cfg)
+    L, ref, xp, xp_ref = run_permute_bf16(s, W.tokens(s))
+    assert np.array_equal(dev_u16(xp), xp_ref)
+    check_counters(L, ref)
+
+
+@pytest.mark.parametrize("T,H,E,K,R", [
+    (1, 8, 1, 1, 1), (5, 16, 4, 2, 2), (300, 24, 7, 3, 7), (777, 520, 33, 5, 3),
+    (64, 8200, 16, 4, 4), (2049, 40, 512, 16, 8), (100, 16384, 8, 2, 2)])
+def test_permute_bf16_edge_shapes(T, H, E, K, R):
+    s = W.Spec("edge", T, H, E, K, R, "uniform", seed=5 + T + H)
+    L, ref, xp, xp_ref = run_permute_bf16(s, W.tokens(s))
+    assert np.array_equal(dev_u16(xp), xp_ref)
+    check_counters(L, ref)
+
+
+def test_permute_bf16_strided_rows_and_skew():
+    s = W.config(5).with_(T=3001, H=264)
+    L, ref, xp, xp_ref = run_permute_bf16(s, W.tokens(s), strided=True)
+    assert np.array_equal(dev_u16(xp), xp_ref)
+    check_counters(L, ref)
+
+
+def run_permute_fp8(s, codes_cpu, xs_cpu):
+    ids = W.topk_ids(s)
+    L, _ = run_layout(ids, s.E, s.R)
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    xp = torch.full((L.P_cap, s.H), SENT, dtype=torch.uint8, device=DEV)
+    xps = torch.full((L.P_cap, s.H // 128), -7.0, dtype=torch.float32, device=DEV)
+    st = ops.new_status()
+    ops.moe_dispatch_permute(codes_cpu.to(DEV), L, xp=xp, x_scales=xs_cpu.to(DEV), xp_scales=xps,
+                             status=st)
+    assert ops.read_status(st) == 0
+    xp_ref = np.full((ref.P_cap, s.H), SENT, np.uint8)
+    xps_ref = np.full((ref.P_cap, s.H // 128), -7.0, np.float32)
+    oracle.permute_rows(codes_cpu.numpy(), ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    oracle.permute_rows(xs_cpu.numpy(), ref.dst_row, s.K, ref.counts, ref.offsets, xps_ref)
+    return L, ref, xp, xps, xp_ref, xps_ref
+
+
+@pytest.mark.parametrize("T,H,E,K,R", [(2048, 7168, 256, 8, 8), (333, 384, 12, 3, 4),
+                                       (50, 128, 3, 2, 1)])
+def test_permute_fp8_parity(T, H, E, K, R):
+    s = W.config(3).with_(T=T, H=H, E=E, K=K, R=R)
+    L, ref, xp, xps, xp_ref, xps_ref = run_permute_fp8(s, W.e4m3_codes(s), W.block_scales(s))
+    assert np.array_equal(xp.cpu().numpy(), xp_ref)
+    assert np.array_equal(xps.cpu().numpy().view(np.uint32), xps_ref.view(np.uint32))
+    check_counters(L, ref)
+
+
+def test_permute_fp8_full_prefill_sampled_rows():
+    """Full prefill size (T=32768): every row checked against x through the
+    oracle's own map (row_src), padding rows zero, counters complete."""
+    s = W.config(3)
+    ids = W.topk_ids(s)
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    codes = W.e4m3_codes(s, device=DEV)
+    xs = W.block_scales(s, device=DEV)
+    L, _ = run_layout(ids, s.E, s.R)
+    st = ops.new_status()
+    xp, xps = ops.moe_dispatch_permute(codes, L, x_scales=xs, status=st)
+    assert ops.read_status(st) == 0
+    rs = torch.from_numpy(ref.row_src[:ref.P]).to(DEV).long()
+    real = rs >= 0
+    tok = torch.where(real, rs // s.K, torch.zeros_like(rs))
+    assert torch.equal(xp[:ref.P][real], codes[tok[real]])
+    assert torch.equal(xps[:ref.P][real], xs[tok[real]])
+    assert int(xp[:ref.P][~real].to(torch.int32).sum()) == 0
+    assert float(xps[:ref.P][~real].abs().sum()) == 0.0
+    check_counters(L, ref)
+
+
+# ---------------------------------------------------------- quantiser ----
+@pytest.mark.parametrize("T,H", [(64, 1024), (1000, 7168), (3, 128)])
+def test_quantize_e4m3_parity(T, H):
+    s = W.config(3).with_(T=T, H=H)
+    x = W.tokens(s)
+    q, qs = ops.moe_quantize_e4m3(x.to(DEV))
+    q_ref, s_ref = oracle.quantize_e4m3(W.as_u16(x))
+    assert np.array_equal(qs.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def test_quantize_then_dispatch_fp8_pipeline():
+    """x -> E4M3 codes (+scales) on both sides independently, then the permute;
+    the two pipelines agree byte for byte."""
+    s = W.config(3).with_(T=1500, H=1024, E=40, K=4, R=4)
+    x = W.tokens(s)
+    q, qs = ops.moe_quantize_e4m3(x.to(DEV))
+    q_ref, s_ref = oracle.quantize_e4m3(W.as_u16(x))
+    ids = W.topk_ids(s)
+    L, _ = run_layout(ids, s.E, s.R)
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    xp, xps = ops.moe_dispatch_permute(q, L, x_scales=qs)
+    xp_ref = np.zeros((ref.P_cap, s.H), np.uint8)
+    xps_ref = np.zeros((ref.P_cap, s.H // 128), np.float32)
+    oracle.permute_rows(q_ref, ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    oracle.permute_rows(s_ref, ref.dst_row, s.K, ref.counts, ref.offsets, xps_ref)
+    P = ref.P
+    assert np.array_equal(xp.cpu().numpy()[:P], xp_ref[:P])
+    assert np.array_equal(xps.cpu().numpy()[:P], xps_ref[:P])
