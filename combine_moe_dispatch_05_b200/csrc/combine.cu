@@ -12,12 +12,13 @@
 //
 // B200 design.  All three are HBM-bound gathers / scatters of 16-byte
 // vectors; there is no contraction to put on tensor cores.
-//   * combine / dispatch_bwd: a warp owns a unit = (token, 64-vector column
-//     chunk); lanes 0..K-1 fetch the slot's row index and scale once and
-//     broadcast them with shuffles; every lane then issues all K 16-byte
-//     gathers of its two columns before reducing, so each warp keeps up to
-//     2*K*512 bytes of loads in flight.  The fp32 reduction runs k = 0..K-1
-//     in order with fma, then adds the shared row, then rounds once.
+//   * combine / dispatch_bwd: a 256-thread CTA owns a token row; threads
+//     0..K-1 fetch the next token's row indices and scales into a second
+//     shared buffer while the CTA works on the current one, so index latency
+//     stays off the critical path.  Each thread issues all K 16-byte gathers
+//     of its column (K*16 bytes in flight per thread) before reducing.  The
+//     fp32 reduction runs k = 0..K-1 in order with fma, then adds the shared
+//     row, then rounds once.
 //   * combine_bwd: a 256-thread CTA owns a token row: it reads grad_out[t]
 //     once, gathers the K rows of y, writes the K scaled rows of grad_y and
 //     reduces the K dot products across the CTA in a fixed order
@@ -27,102 +28,93 @@
 namespace moe {
 namespace {
 
-constexpr int kGatherThreads = 256;
-constexpr int kVecPerLane = 2;   // 16-byte columns per lane per unit
 constexpr int kKBatch = 8;       // gathers issued before reducing
 
+#ifndef MOE_GATHER_CTA_THREADS
+#define MOE_GATHER_CTA_THREADS 256
+#endif
+constexpr int kCtaThreads = MOE_GATHER_CTA_THREADS;
+
+// CTA-per-token form of the same reduction: threads 0..K-1 fetch the next
+// token's row indices and scales while the CTA works on the current token
+// (double-buffered in shared memory), so the index latency is hidden.
 template <bool kScaled, bool kShared>
-__global__ void __launch_bounds__(kGatherThreads)
-gather_reduce_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ dst_row,
-                     const float* __restrict__ scales, const uint16_t* __restrict__ shared,
-                     int64_t T, int K, int H, int64_t P_cap, uint16_t* __restrict__ out,
-                     int32_t* status) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp_id = ((int64_t)blockIdx.x * kGatherThreads + threadIdx.x) >> 5;
-  const int64_t n_warps = ((int64_t)gridDim.x * kGatherThreads) >> 5;
+__global__ void __launch_bounds__(kCtaThreads)
+gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ dst_row,
+                         const float* __restrict__ scales, const uint16_t* __restrict__ shared,
+                         int64_t T, int K, int H, int64_t P_cap, uint16_t* __restrict__ out,
+                         int32_t* status) {
+  __shared__ int32_t s_row[2][MOE_MAX_TOPK];
+  __shared__ float s_sc[2][MOE_MAX_TOPK];
+  const int tid = threadIdx.x;
   const int V = H >> 3;
-  constexpr int kUnitVecs = 32 * kVecPerLane;
-  const int units_per_token = (V + kUnitVecs - 1) / kUnitVecs;
-  const int64_t n_units = T * units_per_token;
-
-  for (int64_t u = warp_id; u < n_units; u += n_warps) {
-    const int64_t t = u / units_per_token;
-    const int c = (int)(u - t * units_per_token);
-
-    int my_row = -1;
-    float my_s = 1.0f;
-    if (lane < K) {
-      my_row = __ldg(dst_row + t * K + lane);
-      if (kScaled) my_s = __ldg(scales + t * K + lane);
-      if (my_row != -1 && (my_row < 0 || (int64_t)my_row >= P_cap)) {
+  auto fetch = [&](int64_t t, int buf) {
+    if (tid < K && t < T) {
+      int r = __ldg(dst_row + t * K + tid);
+      if (r != -1 && (r < 0 || (int64_t)r >= P_cap)) {
         record_error(status, MOE_ERR_BOUNDS);
-        my_row = -1;
+        r = -1;
       }
+      s_row[buf][tid] = r;
+      s_sc[buf][tid] = kScaled ? __ldg(scales + t * K + tid) : 1.0f;
     }
-
-    float acc[kVecPerLane][8];
+  };
+  int buf = 0;
+  fetch(blockIdx.x, 0);
+  __syncthreads();
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    fetch(t + gridDim.x, buf ^ 1);
+    for (int vec = tid; vec < V; vec += kCtaThreads) {
+      float acc[8];
 #pragma unroll
-    for (int i = 0; i < kVecPerLane; ++i)
+      for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
-
-    for (int kb = 0; kb < K; kb += kKBatch) {
-      int rows[kKBatch];
-      uint4 v[kKBatch][kVecPerLane];
+      for (int kb = 0; kb < MOE_MAX_TOPK; kb += kKBatch) {
+        if (kb >= K) break;
+        uint4 v[kKBatch];
 #pragma unroll
-      for (int j = 0; j < kKBatch; ++j) {
-        rows[j] = __shfl_sync(0xffffffffu, my_row, (kb + j) & 31);
-        if (kb + j >= K) rows[j] = -1;
-#pragma unroll
-        for (int i = 0; i < kVecPerLane; ++i) {
-          const int vec = c * kUnitVecs + i * 32 + lane;
-          if (rows[j] >= 0 && vec < V)
-            v[j][i] = ld_nc_v4(y + (int64_t)rows[j] * H + (int64_t)vec * 8);
-          else
-            v[j][i] = make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < kKBatch; ++j) {
+          const int k = kb + j;
+          const int r = k < K ? s_row[buf][k] : -1;
+          v[j] = r >= 0 ? ld_nc_v4(y + (int64_t)r * H + (int64_t)vec * 8) : make_uint4(0, 0, 0, 0);
         }
-      }
 #pragma unroll
-      for (int j = 0; j < kKBatch; ++j) {
-        const float s = __shfl_sync(0xffffffffu, my_s, (kb + j) & 31);
-        if (rows[j] < 0) continue;  // an unplaced slot contributes nothing
-#pragma unroll
-        for (int i = 0; i < kVecPerLane; ++i) {
-          const uint32_t w[4] = {v[j][i].x, v[j][i].y, v[j][i].z, v[j][i].w};
+        for (int j = 0; j < kKBatch; ++j) {
+          const int k = kb + j;
+          const int r = k < K ? s_row[buf][k] : -1;
+          if (r < 0) continue;
+          const float sk = s_sc[buf][k];
+          const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             if (kScaled) {
-              acc[i][2 * q] = fmaf(s, bf16_lo(w[q]), acc[i][2 * q]);
-              acc[i][2 * q + 1] = fmaf(s, bf16_hi(w[q]), acc[i][2 * q + 1]);
+              acc[2 * q] = fmaf(sk, bf16_lo(w[q]), acc[2 * q]);
+              acc[2 * q + 1] = fmaf(sk, bf16_hi(w[q]), acc[2 * q + 1]);
             } else {
-              acc[i][2 * q] = __fadd_rn(acc[i][2 * q], bf16_lo(w[q]));
-              acc[i][2 * q + 1] = __fadd_rn(acc[i][2 * q + 1], bf16_hi(w[q]));
+              acc[2 * q] = __fadd_rn(acc[2 * q], bf16_lo(w[q]));
+              acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_hi(w[q]));
             }
           }
         }
       }
-    }
-
-#pragma unroll
-    for (int i = 0; i < kVecPerLane; ++i) {
-      const int vec = c * kUnitVecs + i * 32 + lane;
-      if (vec >= V) continue;
       if (kShared) {
         const uint4 sv = ld_nc_v4(shared + t * H + (int64_t)vec * 8);
         const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          acc[i][2 * q] = __fadd_rn(acc[i][2 * q], bf16_lo(w[q]));
-          acc[i][2 * q + 1] = __fadd_rn(acc[i][2 * q + 1], bf16_hi(w[q]));
+          acc[2 * q] = __fadd_rn(acc[2 * q], bf16_lo(w[q]));
+          acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_hi(w[q]));
         }
       }
       uint4 o;
-      o.x = pack_bf16x2(acc[i][0], acc[i][1]);
-      o.y = pack_bf16x2(acc[i][2], acc[i][3]);
-      o.z = pack_bf16x2(acc[i][4], acc[i][5]);
-      o.w = pack_bf16x2(acc[i][6], acc[i][7]);
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
       st_v4(out + t * H + (int64_t)vec * 8, o);
     }
+    __syncthreads();
+    buf ^= 1;
   }
 }
 
@@ -299,15 +291,13 @@ int launch_gather(int slot, const uint16_t* y, const int32_t* dst_row, const flo
                   const uint16_t* shared, int64_t T, int K, int H, int64_t P_cap, uint16_t* out,
                   int32_t* status, cudaStream_t s) {
   const int dev = moe_host::current_device();
-  auto kern = gather_reduce_kernel<kScaled, kShared>;
-  const int bps = blocks_per_sm(kern, kGatherThreads, dev, g_occ_comb[slot]);
-  const int64_t units = T * (((H >> 3) + 63) / 64);
+  auto kern = gather_reduce_cta_kernel<kScaled, kShared>;
+  const int bps = blocks_per_sm(kern, kCtaThreads, dev, g_occ_comb[slot]);
   int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
-  const int64_t need = (units + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
-  if (grid > need) grid = need;
+  if (grid > T) grid = T;
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, kGatherThreads, 0, s>>>(y, dst_row, scales, shared, T, K, H, P_cap, out,
-                                                 status);
+  kern<<<(unsigned)grid, kCtaThreads, 0, s>>>(y, dst_row, scales, shared, T, K, H, P_cap, out,
+                                              status);
   return moe_host::launch_status();
 }
 

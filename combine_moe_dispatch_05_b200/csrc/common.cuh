@@ -3,7 +3,7 @@
 // Inline PTX wrappers for the Blackwell features the kernels use: mbarrier
 // transaction barriers, non-multicast bulk copies between global and the
 // issuing CTA's own shared memory (cp.async.bulk), the async-proxy fences
-// they need, gpu-scope acquire loads and acq_rel atomics for the
+// they need, gpu-scope acquire loads and release patterns for the
 // chunk-completion counters, and %globaltimer for bounded waits.
 #pragma once
 
@@ -39,15 +39,19 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
-// The writer that completes a chunk publishes it; acq_rel makes every earlier
-// writer's release part of what a reader acquiring the final count observes.
-__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
-               : "=r"(old)
-               : "l"(p), "r"(v)
-               : "memory");
-  return old;
+// Release pattern for the chunk-completion counters: one fence.acq_rel.gpu,
+// then relaxed gpu-scope adds.  Under the PTX memory model, observation order
+// runs through every later atomic add on the same counter, so a consumer whose
+// ld.acquire.gpu reads the final count synchronizes with each writer's fence
+// and sees every row those writers published.  One fence per batch of adds
+// keeps the release off the copy pipeline's critical path (an acq_rel atom per
+// row costs a full fence each).
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+__device__ __forceinline__ void atomic_add_relaxed_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // ----------------------------------------------------------- shared mem --

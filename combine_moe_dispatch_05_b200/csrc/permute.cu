@@ -4,7 +4,7 @@
 // expert-major buffer (expand_x of the torch_npu npu_moe_distribute_combine
 // API), padding rows of each expert's last 128-row M-tile (TEMPO summary,
 // section 1) are zero-filled, and each finished row bumps its tile's
-// chunk-completion counter with atom.acq_rel.gpu.
+// chunk-completion counter behind a gpu-scope release.
 //
 // B200 design.  The work is pure data movement, so it is written as a bulk
 // copy engine rather than as threads moving registers:
@@ -20,17 +20,33 @@
 //     writes the same number of rows whatever the expert skew.
 //   * counters: a row's +1 is released only after its bulk-store group has
 //     completed (cp.async.bulk.wait_group), behind a proxy fence, with a lag
-//     of a few groups so the copy pipeline never drains.  FP8 scale rows are
-//     copied by the 32 lanes with plain stores before the same release.
+//     of a few groups so the copy pipeline never drains.  The release is one
+//     fence.acq_rel.gpu per token followed by relaxed adds (the pull
+//     request's atom.acq_rel.gpu on every add is a full fence per row).  FP8
+//     scale rows are copied by the 32 lanes with plain stores before the
+//     same release.
 #include "common.cuh"
 
 namespace moe {
 namespace {
 
-constexpr uint32_t kMaxChunk = 16384;  // bytes per bulk copy
+#ifndef MOE_PERM_MAX_CHUNK
+#define MOE_PERM_MAX_CHUNK 16384
+#endif
+#ifndef MOE_PERM_REL_LAG
+#define MOE_PERM_REL_LAG 2
+#endif
+#ifndef MOE_PERM_CTAS_PER_SM
+#define MOE_PERM_CTAS_PER_SM 2
+#endif
+#ifndef MOE_PERM_READ_LAG
+#define MOE_PERM_READ_LAG 1
+#endif
+constexpr uint32_t kMaxChunk = MOE_PERM_MAX_CHUNK;  // bytes per bulk copy
 constexpr int kMaxStages = 16;
-constexpr int kRelLag = 2;             // bulk groups kept in flight before a release
-constexpr int kPermCtasPerSm = 2;
+constexpr int kRelLag = MOE_PERM_REL_LAG;          // bulk groups in flight before a release
+constexpr int kReadLag = MOE_PERM_READ_LAG;        // bulk groups still reading before a refill
+constexpr int kPermCtasPerSm = MOE_PERM_CTAS_PER_SM;
 
 struct PermArgs {
   const uint8_t* x;
@@ -145,12 +161,14 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
     mbar_arrive_expect_tx(&bar[s], len);
     bulk_load_g2s(stage0 + (size_t)s * a.stage_bytes, src, len, &bar[s]);
   };
-  // Release +1 for every placed row of token t inside [v0, v1).
+  // Release +1 for every placed row of token t inside [v0, v1).  The caller
+  // has waited for the rows' bulk stores and issued the proxy fence.
   auto release_token = [&](int64_t t) {  // lane 0 only
     const int64_t sa = max(v0, t * a.K), sb = min(sl_end, (t + 1) * a.K);
+    fence_acq_rel_gpu();
     for (int64_t sl = sa; sl < sb; ++sl) {
       const int32_t r = __ldg(a.dst_row + sl);
-      if (r >= 0 && (int64_t)r < a.P_cap) atomic_add_acq_rel_gpu(a.tile_ready + r / kTile, 1u);
+      if (r >= 0 && (int64_t)r < a.P_cap) atomic_add_relaxed_gpu(a.tile_ready + r / kTile, 1u);
     }
   };
 
@@ -201,9 +219,9 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
       }
     }
     if (lane == 0) {
-      bulk_wait_read<1>();  // the stores of unit u-1 have read their stage
-      if (u >= 1 && issued < n_units) {
-        issue_load(issued);  // lands in the stage unit u-1 used: (u-1+S) % S
+      bulk_wait_read<kReadLag>();  // the stores of unit u-kReadLag have read their stage
+      if (u >= kReadLag && issued < n_units) {
+        issue_load(issued);  // lands in the stage unit u-kReadLag used
         ++issued;
       }
     }
@@ -257,6 +275,7 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
       for (int64_t ur = max((int64_t)0, n_units - kRelLag); ur < n_units; ++ur)
         if ((ur % nch) == nch - 1) release_token(unit_token(ur));
       if (q1 > q0) {
+        fence_acq_rel_gpu();
         int e = 0;
         while (e < E - 1 && s_padpref[e + 1] <= q0) ++e;
         int64_t q = q0;
@@ -264,7 +283,7 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
           while (q >= s_padpref[e + 1]) ++e;
           const int64_t q_end = min(q1, (int64_t)s_padpref[e + 1]);
           const int64_t last_row = (int64_t)s_off[e] + s_cnt[e] + (q_end - 1 - s_padpref[e]);
-          atomic_add_acq_rel_gpu(a.tile_ready + last_row / kTile, (uint32_t)(q_end - q));
+          atomic_add_relaxed_gpu(a.tile_ready + last_row / kTile, (uint32_t)(q_end - q));
           q = q_end;
         }
       }

@@ -149,9 +149,10 @@ MOE_API int moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int K, int E
  *   xp        [P_cap, H] of `dtype`, contiguous, 16-byte aligned.
  *   xp_scales fp32 [P_cap, H/128] (E4M3 only; NULL for bf16).
  *   tile_ready (nullable) counters zeroed by the layout call; each finished
- *            row adds 1 to tile_ready[row/128] with atom.add.acq_rel.gpu
- *            after its bytes (and scales) are globally visible, so a tile
- *            whose counter reads 128 with an acquire load is complete.
+ *            row adds 1 to tile_ready[row/128] after its bytes (and scales)
+ *            are globally visible, behind a gpu-scope release (a
+ *            fence.acq_rel.gpu per token, then relaxed atomic adds), so a
+ *            tile whose counter reads 128 with an ld.acquire.gpu is complete.
  * Data errors: MOE_ERR_BOUNDS if a dst_row entry or offset leaves
  *   [0, P_cap) (that write is skipped); MOE_ERR_TIMEOUT if a staged load
  *   did not land within about 2 s.
