@@ -38,6 +38,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "dispatch+combine HBM GB/s and tokens/s on 1 B200; fraction of HBM peak"
+# kernels per step: layout (count + assign), permute, combine [, combine_bwd, dispatch_bwd]
+LAUNCHES_PER_STEP = {False: 6, True: 4}
 CONFIG_INDEX = 2
 FALLBACK_HBM_GBS = 6650.0
 
@@ -302,7 +304,7 @@ def run_ours(args, world, rank, local):
            "phases_us": {p: round(v, 2) for p, v in phase_us.items()},
            "phases_gbs": {p: round(v, 1) for p, v in phase_gbs.items()},
            "roofline": roofline,
-           "gpu_launches": (7 if not args.fwd_only else 5) * args.steps,
+           "gpu_launches": LAUNCHES_PER_STEP[args.fwd_only] * args.steps,
            "clocks": clk.summary()}
 
     if not args.no_e2e:

@@ -19,7 +19,7 @@
 //     of its column (K*16 bytes in flight per thread) before reducing.  The
 //     fp32 reduction runs k = 0..K-1 in order with fma, then adds the shared
 //     row, then rounds once.
-//   * combine_bwd: a 256-thread CTA owns a token row: it reads grad_out[t]
+//   * combine_bwd: a 128-thread CTA owns a token row: it reads grad_out[t]
 //     once, gathers the K rows of y, writes the K scaled rows of grad_y and
 //     reduces the K dot products across the CTA in a fixed order
 //     (deterministic).  The same CTAs then zero the padding rows of grad_y.
@@ -33,17 +33,21 @@ constexpr int kKBatch = 8;       // gathers issued before reducing
 #ifndef MOE_GATHER_CTA_THREADS
 #define MOE_GATHER_CTA_THREADS 256
 #endif
+#ifndef MOE_GATHER_MINB
+#define MOE_GATHER_MINB 1
+#endif
 constexpr int kCtaThreads = MOE_GATHER_CTA_THREADS;
 
 // CTA-per-token form of the same reduction: threads 0..K-1 fetch the next
 // token's row indices and scales while the CTA works on the current token
 // (double-buffered in shared memory), so the index latency is hidden.
 template <bool kScaled, bool kShared>
-__global__ void __launch_bounds__(kCtaThreads)
+__global__ void __launch_bounds__(kCtaThreads, MOE_GATHER_MINB)
 gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ dst_row,
                          const float* __restrict__ scales, const uint16_t* __restrict__ shared,
                          int64_t T, int K, int H, int64_t P_cap, uint16_t* __restrict__ out,
                          int32_t* status) {
+  pdl_begin();
   __shared__ int32_t s_row[2][MOE_MAX_TOPK];
   __shared__ float s_sc[2][MOE_MAX_TOPK];
   const int tid = threadIdx.x;
@@ -118,21 +122,29 @@ gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restri
   }
 }
 
-constexpr int kBwdThreads = 256;
+#ifndef MOE_BWD_THREADS
+#define MOE_BWD_THREADS 128
+#endif
+#ifndef MOE_BWD_MINB
+#define MOE_BWD_MINB 1
+#endif
+constexpr int kBwdThreads = MOE_BWD_THREADS;
 constexpr int kBwdWarps = kBwdThreads / 32;
 
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kBwdThreads, MOE_BWD_MINB)
 combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ y,
                    const float* __restrict__ scales, const int32_t* __restrict__ dst_row,
                    const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
                    int E, int64_t T, int K, int H, int64_t P_cap,
                    uint16_t* __restrict__ grad_y, float* __restrict__ grad_s,
                    int32_t* status) {
+  pdl_begin();
   __shared__ int32_t s_row[MOE_MAX_TOPK];
   __shared__ float s_sc[MOE_MAX_TOPK];
   __shared__ float s_part[kBwdWarps][MOE_MAX_TOPK];
   __shared__ int32_t s_padpref[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_pad_base[MOE_MAX_EXPERTS];
+  __shared__ int32_t s_pad[MOE_MAX_EXPERTS];
   __shared__ int32_t s_warp[kBwdWarps];
   __shared__ int s_bad;
 
@@ -223,38 +235,13 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
   for (int e = tid; e < E; e += kBwdThreads) {
     const int c = __ldg(counts + e);
     const int pad = (__ldg(offsets + e + 1) - __ldg(offsets + e)) - c;
-    if (pad < 0 || pad >= kTile || c < 0) s_bad = 1;
+    const bool ok = pad >= 0 && pad < kTile && c >= 0;
+    if (!ok) s_bad = 1;
     s_pad_base[e] = __ldg(offsets + e) + c;
+    s_pad[e] = ok ? pad : 0;
   }
-  // exclusive prefix of the padding counts (E <= 512: two per thread)
-  {
-    int p[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int e = 2 * tid + i;
-      p[i] = 0;
-      if (e < E) {
-        const int c = __ldg(counts + e);
-        const int pad = (__ldg(offsets + e + 1) - __ldg(offsets + e)) - c;
-        p[i] = (pad >= 0 && pad < kTile) ? pad : 0;
-      }
-    }
-    const int local = p[0] + p[1];
-    const int incl = warp_inclusive_scan(local);
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      const int v = lane < kBwdWarps ? s_warp[lane] : 0;
-      const int wi = warp_inclusive_scan(v);
-      if (lane < kBwdWarps) s_warp[lane] = wi - v;
-    }
-    __syncthreads();
-    const int excl = s_warp[warp] + incl - local;
-    if (2 * tid < E) s_padpref[2 * tid] = excl;
-    if (2 * tid + 1 < E) s_padpref[2 * tid + 1] = excl + p[0];
-    if (2 * tid == E - 1 || 2 * tid + 1 == E - 1) s_padpref[E] = excl + local;
-    __syncthreads();
-  }
+  __syncthreads();
+  block_exclusive_scan(s_pad, E, s_padpref, s_warp);
   if (s_bad || (int64_t)__ldg(offsets + E) > P_cap) {
     if (tid == 0) record_error(status, MOE_ERR_BOUNDS);
     return;
@@ -296,9 +283,8 @@ int launch_gather(int slot, const uint16_t* y, const int32_t* dst_row, const flo
   int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
   if (grid > T) grid = T;
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, kCtaThreads, 0, s>>>(y, dst_row, scales, shared, T, K, H, P_cap, out,
-                                              status);
-  return moe_host::launch_status();
+  return moe_host::launch(kern, dim3((unsigned)grid), dim3(kCtaThreads), 0, s, y, dst_row, scales,
+                          shared, T, K, H, P_cap, out, status);
 }
 
 int check_rows_args(const void* y, const int32_t* dst_row, int64_t T, int K, int H,
@@ -367,9 +353,9 @@ extern "C" int moe_combine_bwd(const void* grad_out, const void* y, const float*
   int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
   const int64_t need = T + (int64_t)(kTile - 1) * E;
   if (grid > need) grid = need;
-  combine_bwd_kernel<<<(unsigned)grid, kBwdThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(grad_out), static_cast<const uint16_t*>(y), scales, dst_row,
-      expert_counts, expert_offsets, E, T, K, H, P_cap, static_cast<uint16_t*>(grad_y),
-      grad_scales, d_status);
-  return moe_host::launch_status();
+  return moe_host::launch(combine_bwd_kernel, dim3((unsigned)grid), dim3(kBwdThreads), 0,
+                          static_cast<cudaStream_t>(stream), static_cast<const uint16_t*>(grad_out),
+                          static_cast<const uint16_t*>(y), scales, dst_row, expert_counts,
+                          expert_offsets, E, T, K, H, P_cap, static_cast<uint16_t*>(grad_y),
+                          grad_scales, d_status);
 }

@@ -10,12 +10,24 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "moe_dispatch.h"
 
 namespace moe {
 
 constexpr int kTile = MOE_TILE_M;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s for any device-side wait
+
+// ------------------------------------------- programmatic dependent launch --
+// Every kernel starts with these two: it lets the next kernel in the stream
+// begin launching, then waits until the previous kernel has finished and its
+// writes are visible.  Stream order of all memory accesses is unchanged; only
+// the launch latency overlaps the previous kernel's tail.
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
 
 // ---------------------------------------------------------------- status --
 __device__ __forceinline__ void record_error(int32_t* status, int code) {
@@ -182,6 +194,39 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
   return v;
 }
 
+// Block-wide exclusive scan of in[0..n) into out[0..n] (out[n] = total); any
+// n >= 0: each thread sums a contiguous run of ceil(n / blockDim.x) items,
+// the runs are scanned across the block, and each thread writes its run's
+// prefixes.  blockDim.x must be a multiple of 32 and at most 1024; s_warp
+// holds blockDim.x / 32 ints.  Every thread of the block must call it.
+__device__ __forceinline__ void block_exclusive_scan(const int* in, int n, int* out,
+                                                     int* s_warp) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = blockDim.x >> 5;
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int b0 = min(n, tid * per), b1 = min(n, b0 + per);
+  int local = 0;
+  for (int i = b0; i < b1; ++i) local += in[i];
+  const int incl = warp_inclusive_scan(local);
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < nw ? s_warp[lane] : 0;
+    const int wi = warp_inclusive_scan(v);
+    if (lane < nw) s_warp[lane] = wi - v;
+  }
+  __syncthreads();
+  int run = s_warp[warp] + incl - local;
+  for (int i = b0; i < b1; ++i) {
+    const int v = in[i];
+    out[i] = run;
+    run += v;
+  }
+  if (b1 == n && b0 < b1) out[n] = run;
+  if (n == 0 && tid == 0) out[0] = 0;
+  __syncthreads();
+}
+
 }  // namespace moe
 
 // ------------------------------------------------------------ host side --
@@ -192,6 +237,25 @@ int current_device();
 int launch_status();  // MOE_OK or MOE_ERR_CUDA from cudaGetLastError()
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Launches with programmatic stream serialization allowed (see pdl_begin).
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+           Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 }  // namespace moe_host

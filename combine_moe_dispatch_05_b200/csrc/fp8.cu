@@ -19,6 +19,7 @@ constexpr int kQThreads = 256;
 __global__ void __launch_bounds__(kQThreads)
 quantize_e4m3_kernel(const uint16_t* __restrict__ x, int64_t T, int H, int64_t stride,
                      uint8_t* __restrict__ q, float* __restrict__ qs) {
+  pdl_begin();
   const int nb = H / 128;
   const int64_t n_units = T * nb;
   const int lane = threadIdx.x & 31, sub = lane & 15;
@@ -80,8 +81,7 @@ extern "C" int moe_quantize_e4m3(const void* x, int64_t T, int H, int64_t x_row_
   int64_t grid = (units * 16 + moe::kQThreads - 1) / moe::kQThreads;
   const int64_t cap = (int64_t)moe_host::sm_count(dev) * 8;
   if (grid > cap) grid = cap;
-  moe::quantize_e4m3_kernel<<<(unsigned)grid, moe::kQThreads, 0,
-                              static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(x), T, H, x_row_stride, static_cast<uint8_t*>(q), q_scales);
-  return moe_host::launch_status();
+  return moe_host::launch(moe::quantize_e4m3_kernel, dim3((unsigned)grid), dim3(moe::kQThreads), 0,
+                          static_cast<cudaStream_t>(stream), static_cast<const uint16_t*>(x), T, H,
+                          x_row_stride, static_cast<uint8_t*>(q), q_scales);
 }

@@ -90,6 +90,7 @@ __device__ __forceinline__ int64_t checked_row(const PermArgs& a, int64_t slot) 
 }
 
 __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
+  pdl_begin();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_cnt[MOE_MAX_EXPERTS];
@@ -366,6 +367,6 @@ extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
   const int64_t by_work = (v_bound + 7) / 8;
   if (grid > by_work) grid = by_work;
   if (grid < 1) grid = 1;
-  permute_kernel<<<(unsigned)grid, 32, dyn, static_cast<cudaStream_t>(stream)>>>(a);
-  return moe_host::launch_status();
+  return moe_host::launch(permute_kernel, dim3((unsigned)grid), dim3(32), dyn,
+                          static_cast<cudaStream_t>(stream), a);
 }

@@ -27,6 +27,7 @@ tile_checksum_kernel(const uint32_t* tile_ready, const int32_t* __restrict__ off
                      const uint8_t* xp, int64_t row_bytes, const float* xs, int scale_cols,
                      int64_t P_cap, uint32_t* __restrict__ checksums, int64_t timeout_ns,
                      int32_t* status) {
+  pdl_begin();
   __shared__ int s_ok;
   __shared__ uint32_t s_red[kConsThreads / 32];
   const int tid = threadIdx.x;
@@ -99,9 +100,8 @@ extern "C" int moe_wait_tiles_checksum(const uint32_t* tile_ready, const int32_t
   int64_t grid = (int64_t)moe_host::sm_count(dev) * 4;
   if (grid > max_tiles) grid = max_tiles;
   if (grid < 1) grid = 1;
-  moe::tile_checksum_kernel<<<(unsigned)grid, moe::kConsThreads, 0,
-                              static_cast<cudaStream_t>(stream)>>>(
-      tile_ready, expert_offsets, E, static_cast<const uint8_t*>(xp), row_bytes, xp_scales,
-      scale_cols, P_cap, checksums, timeout_ns, d_status);
-  return moe_host::launch_status();
+  return moe_host::launch(moe::tile_checksum_kernel, dim3((unsigned)grid), dim3(moe::kConsThreads),
+                          0, static_cast<cudaStream_t>(stream), tile_ready, expert_offsets, E,
+                          static_cast<const uint8_t*>(xp), row_bytes, xp_scales, scale_cols, P_cap,
+                          checksums, timeout_ns, d_status);
 }

@@ -157,7 +157,8 @@ def test_backward_parity_workloads(cfg):
 
 
 @pytest.mark.parametrize("T,H,E,K,R", [(1, 8, 1, 1, 1), (77, 24, 6, 3, 2), (300, 1032, 40, 16, 4),
-                                       (2, 7168, 256, 8, 8)])
+                                       (2, 7168, 256, 8, 8), (1000, 64, 512, 16, 8),
+                                       (500, 40, 37, 3, 1), (129, 7176, 300, 2, 2)])
 def test_backward_parity_edge_shapes(T, H, E, K, R):
     s = W.Spec("edge", T, H, E, K, R, "uniform", seed=11 + T + H)
     check_combine_bwd(s)
