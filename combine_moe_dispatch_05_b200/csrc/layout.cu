@@ -272,3 +272,51 @@ extern "C" int moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int K, in
                           tpb, expert_counts, expert_offsets, rank_counts, rank_offsets, dst_row,
                           row_src, P_cap, d_status);
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free layout: the same two kernels, with their scratch in a
+// file-scope device array instead of a caller-provided workspace.  Callers
+// that cannot allocate device memory at call time use this one (see the
+// header).  In host code the array's name is only a host-side stand-in, so
+// each device's real address is looked up once, with that device current.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+static __device__ __align__(256) unsigned char g_layout_scratch[MOE_LAYOUT_STATIC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_layout_scratch_mu;
+void* g_layout_scratch_ptr[64] = {};
+}  // namespace
+
+extern "C" int moe_dispatch_layout_static(const int32_t* topk_idx, int64_t T, int K, int E,
+                                          int R, int32_t* expert_counts,
+                                          int32_t* expert_offsets, int32_t* rank_counts,
+                                          int32_t* rank_offsets, int32_t* dst_row,
+                                          int32_t* row_src, uint32_t* tile_ready,
+                                          int64_t P_cap, int32_t* d_status, void* stream) {
+  const size_t need = moe_layout_workspace_bytes(T, K, E);
+  if (need == (size_t)-1) return MOE_ERR_INVALID_ARG;
+  if (need > (size_t)MOE_LAYOUT_STATIC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_layout_scratch_mu);
+    if (g_layout_scratch_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_layout_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+      }
+      g_layout_scratch_ptr[dev] = p;
+    }
+    scratch = g_layout_scratch_ptr[dev];
+  }
+  return moe_dispatch_layout(topk_idx, T, K, E, R, expert_counts, expert_offsets, rank_counts,
+                             rank_offsets, dst_row, row_src, tile_ready, P_cap, d_status,
+                             scratch, (size_t)MOE_LAYOUT_STATIC_SCRATCH_BYTES, stream);
+}

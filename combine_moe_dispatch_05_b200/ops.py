@@ -32,6 +32,8 @@ SIGNATURES = {
     "moe_layout_workspace_bytes": (_sz, [_i64, _int, _int]),
     "moe_dispatch_layout": (_int, [_vp, _i64, _int, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _i64, _vp, _vp, _sz, _vp]),
+    "moe_dispatch_layout_static": (_int, [_vp, _i64, _int, _int, _int, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _vp, _i64, _vp, _vp]),
     "moe_dispatch_permute": (_int, [_vp, _int, _i64, _int, _i64, _vp, _i64, _vp, _int, _vp, _vp,
                                     _int, _vp, _vp, _i64, _vp, _vp, _vp]),
     "moe_combine": (_int, [_vp, _vp, _vp, _vp, _i64, _int, _int, _i64, _vp, _vp, _vp]),
@@ -172,6 +174,25 @@ def moe_dispatch_layout(topk_idx: torch.Tensor, E: int, R: int, layout: Optional
         _ptr(L.tile_ready), L.P_cap, _ptr(status), _ptr(L.workspace), L.workspace.numel(),
         _stream(stream))
     _check(rc, "moe_dispatch_layout")
+    return L
+
+
+def moe_dispatch_layout_static(topk_idx: torch.Tensor, E: int, R: int,
+                               layout: Optional[Layout] = None,
+                               status: Optional[torch.Tensor] = None,
+                               P_cap: Optional[int] = None, stream=None) -> Layout:
+    """moe_dispatch_layout without a workspace, for callers that cannot
+    allocate device memory at call time: the library's own static scratch is
+    used.  Outputs are still the caller's (pass ``layout`` to avoid any
+    allocation here as well)."""
+    _cuda(topk_idx, "topk_idx", torch.int32)
+    T, K = topk_idx.shape
+    L = layout or alloc_layout(T, K, E, R, topk_idx.device, P_cap)
+    rc = lib().moe_dispatch_layout_static(
+        _ptr(topk_idx), T, K, E, R, _ptr(L.expert_counts), _ptr(L.expert_offsets),
+        _ptr(L.rank_counts), _ptr(L.rank_offsets), _ptr(L.dst_row), _ptr(L.row_src),
+        _ptr(L.tile_ready), L.P_cap, _ptr(status), _stream(stream))
+    _check(rc, "moe_dispatch_layout_static")
     return L
 
 

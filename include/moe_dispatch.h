@@ -133,6 +133,41 @@ MOE_API int moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int K, int E
                         void* stream);
 
 /*
+ * Allocation-free form of moe_dispatch_layout.  The pages have no
+ * counterpart; this exists for callers that cannot allocate device memory
+ * when they call: engines whose device memory is planned once at start-up
+ * and may not grow, foreign-language callers with no device allocator at
+ * hand, and hot paths that must not pay for cudaMalloc, which can
+ * synchronise the whole device.
+ *
+ * Same arguments, outputs and results as moe_dispatch_layout, minus the
+ * workspace: the scratch lives in a static device array of
+ * MOE_LAYOUT_STATIC_SCRATCH_BYTES that is part of the library image, so every
+ * GPU that loads the library holds it until the process exits.  The call
+ * makes no allocation of any kind.
+ *   - Sizes: accepted while moe_layout_workspace_bytes(T, K, E) is at most
+ *     MOE_LAYOUT_STATIC_SCRATCH_BYTES (for E=256, K=8: up to 116480 tokens);
+ *     larger sizes return MOE_ERR_UNSUPPORTED before anything is launched.
+ *   - Set-up: the first call on each device looks up that device's address
+ *     of the array (cudaGetSymbolAddress, with the device current); make
+ *     that first call before any stream capture.  A failed lookup returns
+ *     MOE_ERR_CUDA.
+ *   - Sharing: all calls on a device use the same array, which keeps the last
+ *     call's contents.  Nothing in it needs to start at zero (every word the
+ *     kernels read is written earlier in the same call), but calls that may
+ *     overlap on the GPU (different streams without ordering between them)
+ *     race on it; order them, or use moe_dispatch_layout with separate
+ *     workspaces.
+ */
+#define MOE_LAYOUT_STATIC_SCRATCH_BYTES (4u << 20)
+MOE_API int moe_dispatch_layout_static(const int32_t* topk_idx, int64_t T, int K, int E, int R,
+                                       int32_t* expert_counts, int32_t* expert_offsets,
+                                       int32_t* rank_counts, int32_t* rank_offsets,
+                                       int32_t* dst_row, int32_t* row_src,
+                                       uint32_t* tile_ready, int64_t P_cap, int32_t* d_status,
+                                       void* stream);
+
+/*
  * Dispatch permute (the fused unzip of [DEP]; produces [ASC] expand_x).
  *   xp[dst_row[t*K+k]] = x[t]  for every placed slot, byte for byte;
  *   padding rows [offsets[e] + counts[e], offsets[e+1]) = 0 (E4M3: code
