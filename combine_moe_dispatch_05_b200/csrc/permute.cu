@@ -15,9 +15,11 @@
 //     bytes, one per destination row.  The row is read from HBM once and
 //     never passes through registers.
 //   * padding rows are bulk-stored from a zero-filled shared chunk.
-//   * work is split by "virtual rows": the T*K slots followed by the
-//     padding rows, cut into equal contiguous ranges per CTA, so every CTA
-//     writes the same number of rows whatever the expert skew.
+//   * every CTA takes an equal contiguous run of the T*K slots and an equal
+//     run of the padding rows, so each writes the same number of rows of
+//     each kind whatever the expert skew; a CTA's padding rows are issued a
+//     few at a time ahead of each token unit's load wait, which keeps the
+//     copy engine busy while the load is in flight.
 //   * counters: a row's +1 is released only after its bulk-store group has
 //     completed (cp.async.bulk.wait_group), behind a proxy fence, with a lag
 //     of a few groups so the copy pipeline never drains.  The release is one
@@ -131,12 +133,12 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
   }
   __syncwarp();
 
-  // ---- this CTA's share of the virtual rows ----
+  // ---- this CTA's share: an equal run of slots and an equal run of padding rows ----
   const int64_t TK = a.T * a.K;
-  const int64_t V = TK + run;
-  const int64_t G = gridDim.x;
-  const int64_t v0 = V * blockIdx.x / G;
-  const int64_t v1 = V * (blockIdx.x + 1) / G;
+  const int64_t PAD = run;
+  const int64_t G = gridDim.x, c = blockIdx.x;
+  const int64_t s0 = TK * c / G, s1 = TK * (c + 1) / G;      // slots
+  const int64_t q0 = PAD * c / G, q1 = PAD * (c + 1) / G;    // padding indices
 
   // ---- ring set-up ----
   for (uint32_t i = lane * 16; i < a.stage_bytes; i += 32 * 16)
@@ -149,9 +151,13 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
   __syncwarp();
 
   const int nch = a.n_chunks;
-  const int64_t sl_end = v1 < TK ? v1 : TK;
-  const int64_t t_first = v0 < sl_end ? v0 / a.K : 0;
-  const int64_t n_units = v0 < sl_end ? ((sl_end - 1) / a.K - t_first + 1) * nch : 0;
+  const int64_t t_first = s0 < s1 ? s0 / a.K : 0;
+  const int64_t n_units = s0 < s1 ? ((s1 - 1) / a.K - t_first + 1) * nch : 0;
+  // padding rows issued alongside unit u: [pad_lo(u), pad_lo(u + 1)); all of
+  // them at once when this CTA has no token units
+  auto pad_lo = [&](int64_t u) {
+    return n_units > 0 ? q0 + (q1 - q0) * u / n_units : (u > 0 ? q1 : q0);
+  };
 
   auto unit_token = [&](int64_t u) { return t_first + u / nch; };
   auto issue_load = [&](int64_t u) {  // lane 0 only
@@ -162,15 +168,62 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
     mbar_arrive_expect_tx(&bar[s], len);
     bulk_load_g2s(stage0 + (size_t)s * a.stage_bytes, src, len, &bar[s]);
   };
-  // Release +1 for every placed row of token t inside [v0, v1).  The caller
-  // has waited for the rows' bulk stores and issued the proxy fence.
-  auto release_token = [&](int64_t t) {  // lane 0 only
-    const int64_t sa = max(v0, t * a.K), sb = min(sl_end, (t + 1) * a.K);
-    fence_acq_rel_gpu();
-    for (int64_t sl = sa; sl < sb; ++sl) {
-      const int32_t r = __ldg(a.dst_row + sl);
-      if (r >= 0 && (int64_t)r < a.P_cap) atomic_add_relaxed_gpu(a.tile_ready + r / kTile, 1u);
+
+  // Walks padding indices in increasing order and yields their rows.
+  struct PadCursor {
+    int e;
+    __device__ void seek(const int32_t* padpref, int E, int64_t q) {
+      int lo = 0, hi = E - 1;  // last expert with padpref <= q
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (padpref[mid] <= q) lo = mid; else hi = mid - 1;
+      }
+      e = lo;
     }
+  };
+  PadCursor issue_cur, rel_cur;
+  issue_cur.seek(s_padpref, E, q0);
+  rel_cur.e = issue_cur.e;
+  auto pad_row = [&](PadCursor& cur, int64_t q) -> int64_t {
+    while (q >= s_padpref[cur.e + 1]) ++cur.e;
+    return (int64_t)s_off[cur.e] + s_cnt[cur.e] + (q - s_padpref[cur.e]);
+  };
+  // zero rows for padding indices [qa, qb): lanes clear the scale rows, lane 0
+  // bulk-stores the zero chunk over every chunk of each row
+  auto issue_padding = [&](int64_t qa, int64_t qb) {
+    for (int64_t q = qa; q < qb; ++q) {
+      const int64_t r = pad_row(issue_cur, q);
+      if (a.scale_cols > 0)
+        for (int cc = lane; cc < a.scale_cols; cc += 32) a.xp_scales[r * a.scale_cols + cc] = 0.0f;
+      if (lane == 0)
+        for (int ch = 0; ch < nch; ++ch)
+          bulk_store_s2g(a.xp + r * a.row_bytes + (int64_t)ch * a.chunk_cap, zero, chunk_len(a, ch));
+    }
+  };
+  // +n for padding indices [qa, qb), one add per run inside one expert (all
+  // padding rows of an expert share its last tile)
+  auto release_padding = [&](int64_t qa, int64_t qb) {  // lane 0 only, after the fence
+    int64_t q = qa;
+    while (q < qb) {
+      const int64_t r = pad_row(rel_cur, q);
+      const int64_t q_end = min(qb, (int64_t)s_padpref[rel_cur.e + 1]);
+      atomic_add_relaxed_gpu(a.tile_ready + r / kTile, (uint32_t)(q_end - q));
+      q = q_end;
+    }
+  };
+  // Release the rows whose bulk-store group belonged to unit ur: the token's
+  // slots (after its last chunk) and the padding rows issued with the unit.
+  auto release_unit = [&](int64_t ur) {  // lane 0 only
+    fence_acq_rel_gpu();
+    if ((ur % nch) == nch - 1) {
+      const int64_t t = unit_token(ur);
+      const int64_t sa = max(s0, t * a.K), sb = min(s1, (t + 1) * a.K);
+      for (int64_t sl = sa; sl < sb; ++sl) {
+        const int32_t r = __ldg(a.dst_row + sl);
+        if (r >= 0 && (int64_t)r < a.P_cap) atomic_add_relaxed_gpu(a.tile_ready + r / kTile, 1u);
+      }
+    }
+    release_padding(pad_lo(ur), pad_lo(ur + 1));
   };
 
   int64_t issued = 0;
@@ -181,6 +234,8 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
   for (int64_t u = 0; u < n_units; ++u) {
     const int s = (int)(u % S);
     const uint32_t parity = (uint32_t)((u / S) & 1);
+    // padding first: it needs no load, so it keeps the copy engine busy
+    issue_padding(pad_lo(u), pad_lo(u + 1));
     int ok = 1;
     if (lane == 0) ok = mbar_wait_bounded(&bar[s], parity) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -190,14 +245,14 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
     }
     const int64_t t = unit_token(u);
     const int ch = (int)(u % nch);
-    const int64_t sa = max(v0, t * a.K), sb = min(sl_end, (t + 1) * a.K);
+    const int64_t sa = max(s0, t * a.K), sb = min(s1, (t + 1) * a.K);
 
     if (ch == 0 && a.scale_cols > 0) {  // FP8 scale row, all lanes
       for (int64_t sl = sa; sl < sb; ++sl) {
         const int64_t r = checked_row(a, sl);
         if (r < 0) continue;
-        for (int c = lane; c < a.scale_cols; c += 32)
-          a.xp_scales[r * a.scale_cols + c] = __ldg(a.x_scales + t * a.xs_stride + c);
+        for (int cc = lane; cc < a.scale_cols; cc += 32)
+          a.xp_scales[r * a.scale_cols + cc] = __ldg(a.x_scales + t * a.xs_stride + cc);
       }
     }
     if (lane == 0) {
@@ -211,12 +266,11 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
       bulk_commit();
     }
     if (a.tile_ready) {
-      __syncwarp();  // scale stores of the lanes precede lane 0's release
+      __syncwarp();  // the lanes' scale stores precede lane 0's release
       if (lane == 0) {
         bulk_wait_all<kRelLag>();  // groups <= u - kRelLag have completed
         fence_proxy_async_global();
-        const int64_t ur = u - kRelLag;
-        if (ur >= 0 && (ur % nch) == nch - 1) release_token(unit_token(ur));
+        if (u >= kRelLag) release_unit(u - kRelLag);
       }
     }
     if (lane == 0) {
@@ -239,32 +293,9 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
     }
     return;
   }
-
-  // ---- padding rows of this range: zero bytes (and zero scales) ----
-  const int64_t q0 = max(v0, TK) - TK, q1 = v1 - TK;
-  if (q1 > q0) {
-    // expert holding padding index q0
-    int e = 0;
-    {
-      int lo = 0, hi = E - 1;  // last e with padpref[e] <= q0
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_padpref[mid] <= q0) lo = mid; else hi = mid - 1;
-      }
-      e = lo;
-    }
-    for (int64_t q = q0; q < q1; ++q) {
-      while (q >= s_padpref[e + 1]) ++e;
-      const int64_t r = (int64_t)s_off[e] + s_cnt[e] + (q - s_padpref[e]);
-      if (a.scale_cols > 0)
-        for (int c = lane; c < a.scale_cols; c += 32) a.xp_scales[r * a.scale_cols + c] = 0.0f;
-      if (lane == 0) {
-        for (int ch = 0; ch < nch; ++ch)
-          bulk_store_s2g(a.xp + r * a.row_bytes + (int64_t)ch * a.chunk_cap, zero,
-                         chunk_len(a, ch));
-        bulk_commit();
-      }
-    }
+  if (n_units == 0) {  // no token rows here: all of this CTA's padding at once
+    issue_padding(q0, q1);
+    if (lane == 0) bulk_commit();
   }
 
   // ---- drain, then release what is still pending ----
@@ -273,20 +304,11 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
     bulk_wait_all<0>();
     if (a.tile_ready) {
       fence_proxy_async_global();
-      for (int64_t ur = max((int64_t)0, n_units - kRelLag); ur < n_units; ++ur)
-        if ((ur % nch) == nch - 1) release_token(unit_token(ur));
-      if (q1 > q0) {
+      if (n_units > 0) {
+        for (int64_t ur = max((int64_t)0, n_units - kRelLag); ur < n_units; ++ur) release_unit(ur);
+      } else {
         fence_acq_rel_gpu();
-        int e = 0;
-        while (e < E - 1 && s_padpref[e + 1] <= q0) ++e;
-        int64_t q = q0;
-        while (q < q1) {
-          while (q >= s_padpref[e + 1]) ++e;
-          const int64_t q_end = min(q1, (int64_t)s_padpref[e + 1]);
-          const int64_t last_row = (int64_t)s_off[e] + s_cnt[e] + (q_end - 1 - s_padpref[e]);
-          atomic_add_relaxed_gpu(a.tile_ready + last_row / kTile, (uint32_t)(q_end - q));
-          q = q_end;
-        }
+        release_padding(q0, q1);
       }
     }
   }
