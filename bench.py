@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--fwd-only", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the per-call timings of the other workloads")
     return ap.parse_args()
 
 
@@ -307,6 +309,9 @@ def run_ours(args, world, rank, local):
            "gpu_launches": LAUNCHES_PER_STEP[args.fwd_only] * args.steps,
            "clocks": clk.summary()}
 
+    if not args.no_extra and world == 1:
+        res["other_workloads"] = extra_workloads(args, dev, flush, stream)
+
     if not args.no_e2e:
         res["e2e"] = e2e(args, ops, torch, dev, stream, L, (ids_h, sc_h, x_h, g_h),
                          (ids, sc, x, g), (xp, out, gy, gs, gx, st), flush, T, K, E, R,
@@ -412,6 +417,123 @@ def e2e(args, ops, torch, dev, stream, L, host_in, dev_in, bufs, flush, T, K, E,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "overlap": "copies on separate streams, two alternating buffer sets",
             "l2": "not flushed: each step moves ~3.2 GB through HBM, far beyond L2"}
+
+
+# ------------------------------------------------------ other workloads --
+def time_calls(torch, calls, flush, steps, stream):
+    """Median device time (us) of each call, L2 flushed before each."""
+    out = {}
+    for name, fn in calls:
+        for _ in range(3):
+            flush.zero_()
+            fn()
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        out[name] = statistics.median(ts)
+    return out
+
+
+def extra_workloads(args, dev, flush, stream):
+    """Per-call device times on the other workloads (prefill FP8 dispatch,
+    shared-expert combine, skewed backward), reported beside the step."""
+    import torch
+    from combine_moe_dispatch_05_b200 import ops
+    from combine_moe_dispatch_05_b200 import workloads as W
+    steps = 10
+    res = {}
+
+    # prefill: FP8 dispatch (quantise then permute, and the fused call), bf16 combine
+    s = W.config(3)
+    T, H, E, K, R = s.T, s.H, s.E, s.K, s.R
+    ids = W.topk_ids(s).to(dev)
+    x = W.tokens(s, device=dev)
+    L = ops.moe_dispatch_layout(ids, E, R)
+    q, qs = ops.moe_quantize_e4m3(x)
+    xp, xps = ops.moe_dispatch_permute(q, L, x_scales=qs)
+    y = W.expert_out(s, L.P_cap, device=dev)
+    sc = W.topk_scales(s).to(dev)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+    P = int(L.expert_offsets[E])
+    nb = H // 128
+    t = time_calls(torch, [
+        ("layout", lambda: ops.moe_dispatch_layout(ids, E, R, layout=L)),
+        ("quantize", lambda: ops.moe_quantize_e4m3(x, q=q, q_scales=qs)),
+        ("permute_e4m3", lambda: ops.moe_dispatch_permute(q, L, xp=xp, x_scales=qs,
+                                                          xp_scales=xps)),
+        ("permute_quant_fused", lambda: ops.moe_dispatch_permute_quant(x, L, xp=xp,
+                                                                       xp_scales=xps)),
+        ("combine", lambda: ops.moe_combine(y, L.dst_row, sc, out=out)),
+    ], flush, steps, stream)
+    b = {"layout": 8 * T * K + 4 * P, "quantize": 2 * T * H + T * H + 4 * T * nb,
+         "permute_e4m3": T * H + 4 * T * nb + P * H + 4 * P * nb,
+         "permute_quant_fused": 2 * T * H + P * H + 4 * P * nb,
+         "combine": 2 * T * K * H + 8 * T * K + 2 * T * H}
+    res[s.name] = {"T": T, "H": H, "E": E, "K": K, "P": P,
+                   "us": {k: round(v, 1) for k, v in t.items()},
+                   "GBps": {k: round(b[k] / (t[k] * 1e-6) / 1e9, 1) for k in t},
+                   "dispatch_unfused_us": round(t["quantize"] + t["permute_e4m3"], 1),
+                   "dispatch_fused_us": round(t["permute_quant_fused"], 1)}
+    del x, q, qs, xp, xps, y, out, L
+    torch.cuda.empty_cache()
+
+    # shared expert: bf16 dispatch + combine with the unweighted shared term
+    s = W.config(4)
+    T, H, E, K, R = s.T, s.H, s.E, s.K, s.R
+    ids = W.topk_ids(s).to(dev)
+    x = W.tokens(s, device=dev)
+    L = ops.moe_dispatch_layout(ids, E, R)
+    xp = ops.moe_dispatch_permute(x, L)
+    y = W.expert_out(s, L.P_cap, device=dev)
+    sh = W.shared_out(s, device=dev)
+    sc = W.topk_scales(s).to(dev)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+    P = int(L.expert_offsets[E])
+    t = time_calls(torch, [
+        ("layout", lambda: ops.moe_dispatch_layout(ids, E, R, layout=L)),
+        ("permute", lambda: ops.moe_dispatch_permute(x, L, xp=xp)),
+        ("combine_shared", lambda: ops.moe_combine(y, L.dst_row, sc, shared_x=sh, out=out)),
+    ], flush, steps, stream)
+    b = {"layout": 8 * T * K + 4 * P, "permute": 2 * T * H + 2 * P * H,
+         "combine_shared": 2 * T * K * H + 8 * T * K + 4 * T * H}
+    res[s.name] = {"T": T, "H": H, "E": E, "K": K, "P": P,
+                   "us": {k: round(v, 1) for k, v in t.items()},
+                   "GBps": {k: round(b[k] / (t[k] * 1e-6) / 1e9, 1) for k in t}}
+    del x, xp, y, sh, out, L
+    torch.cuda.empty_cache()
+
+    # backward under skew (hot expert in 60% of tokens)
+    s = W.config(5)
+    T, H, E, K, R = s.T, s.H, s.E, s.K, s.R
+    ids = W.topk_ids(s).to(dev)
+    L = ops.moe_dispatch_layout(ids, E, R)
+    y = W.expert_out(s, L.P_cap, device=dev)
+    g = W.grad_out(s, device=dev)
+    sc = W.topk_scales(s).to(dev)
+    gy = torch.empty_like(y)
+    gs = torch.empty((T, K), dtype=torch.float32, device=dev)
+    gx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+    P = int(L.expert_offsets[E])
+    t = time_calls(torch, [
+        ("layout", lambda: ops.moe_dispatch_layout(ids, E, R, layout=L)),
+        ("combine_bwd", lambda: ops.moe_combine_bwd(g, y, sc, L, grad_y=gy, grad_scales=gs)),
+        ("dispatch_bwd", lambda: ops.moe_dispatch_bwd(gy, L.dst_row, T, K, grad_x=gx)),
+    ], flush, steps, stream)
+    b = {"layout": 8 * T * K + 4 * P, "combine_bwd": 2 * T * H + 2 * T * K * H + 2 * P * H + 12 * T * K,
+         "dispatch_bwd": 2 * T * K * H + 2 * T * H + 4 * T * K}
+    res[s.name] = {"T": T, "H": H, "E": E, "K": K, "P": P,
+                   "us": {k: round(v, 1) for k, v in t.items()},
+                   "GBps": {k: round(b[k] / (t[k] * 1e-6) / 1e9, 1) for k in t}}
+    return res
 
 
 # --------------------------------------------------------- oracle timing --

@@ -38,16 +38,20 @@ constexpr int kKBatch = 8;       // gathers issued before reducing
 #endif
 constexpr int kCtaThreads = MOE_GATHER_CTA_THREADS;
 
-// CTA-per-token form of the same reduction: threads 0..K-1 fetch the next
-// token's row indices and scales while the CTA works on the current token
-// (double-buffered in shared memory), so the index latency is hidden.
-template <bool kScaled, bool kShared>
+// CTA-per-token reduction: threads 0..K-1 fetch the next token's row indices
+// and scales while the CTA works on the current token (double-buffered in
+// shared memory), so index latency stays off the critical path.  Each thread
+// handles kU columns at a time and issues kU * min(K, 8 / kU) 16-byte gathers
+// before reducing, so about eight loads are in flight per thread whatever K
+// is (kU = 8 / K rounded down to a power of two).
+template <bool kScaled, bool kShared, int kU>
 __global__ void __launch_bounds__(kCtaThreads, MOE_GATHER_MINB)
 gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ dst_row,
                          const float* __restrict__ scales, const uint16_t* __restrict__ shared,
                          int64_t T, int K, int H, int64_t P_cap, uint16_t* __restrict__ out,
                          int32_t* status) {
   pdl_begin();
+  constexpr int kKB = kKBatch / kU;  // rows per batch
   __shared__ int32_t s_row[2][MOE_MAX_TOPK];
   __shared__ float s_sc[2][MOE_MAX_TOPK];
   const int tid = threadIdx.x;
@@ -68,54 +72,67 @@ gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restri
   __syncthreads();
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     fetch(t + gridDim.x, buf ^ 1);
-    for (int vec = tid; vec < V; vec += kCtaThreads) {
-      float acc[8];
+    for (int vb = tid; vb < V; vb += kCtaThreads * kU) {
+      float acc[kU][8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+      for (int i = 0; i < kU; ++i)
 #pragma unroll
-      for (int kb = 0; kb < MOE_MAX_TOPK; kb += kKBatch) {
-        if (kb >= K) break;
-        uint4 v[kKBatch];
+        for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
+      for (int kb = 0; kb < K; kb += kKB) {
+        uint4 v[kKB][kU];
 #pragma unroll
-        for (int j = 0; j < kKBatch; ++j) {
+        for (int j = 0; j < kKB; ++j) {
           const int k = kb + j;
           const int r = k < K ? s_row[buf][k] : -1;
-          v[j] = r >= 0 ? ld_nc_v4(y + (int64_t)r * H + (int64_t)vec * 8) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int i = 0; i < kU; ++i) {
+            const int vec = vb + i * kCtaThreads;
+            v[j][i] = (r >= 0 && vec < V) ? ld_nc_v4(y + (int64_t)r * H + (int64_t)vec * 8)
+                                          : make_uint4(0, 0, 0, 0);
+          }
         }
 #pragma unroll
-        for (int j = 0; j < kKBatch; ++j) {
+        for (int j = 0; j < kKB; ++j) {
           const int k = kb + j;
           const int r = k < K ? s_row[buf][k] : -1;
-          if (r < 0) continue;
+          if (r < 0) continue;  // an unplaced slot contributes nothing
           const float sk = s_sc[buf][k];
-          const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (kScaled) {
-              acc[2 * q] = fmaf(sk, bf16_lo(w[q]), acc[2 * q]);
-              acc[2 * q + 1] = fmaf(sk, bf16_hi(w[q]), acc[2 * q + 1]);
-            } else {
-              acc[2 * q] = __fadd_rn(acc[2 * q], bf16_lo(w[q]));
-              acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_hi(w[q]));
+          for (int i = 0; i < kU; ++i) {
+            const uint32_t w[4] = {v[j][i].x, v[j][i].y, v[j][i].z, v[j][i].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (kScaled) {
+                acc[i][2 * q] = fmaf(sk, bf16_lo(w[q]), acc[i][2 * q]);
+                acc[i][2 * q + 1] = fmaf(sk, bf16_hi(w[q]), acc[i][2 * q + 1]);
+              } else {
+                acc[i][2 * q] = __fadd_rn(acc[i][2 * q], bf16_lo(w[q]));
+                acc[i][2 * q + 1] = __fadd_rn(acc[i][2 * q + 1], bf16_hi(w[q]));
+              }
             }
           }
         }
       }
-      if (kShared) {
-        const uint4 sv = ld_nc_v4(shared + t * H + (int64_t)vec * 8);
-        const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          acc[2 * q] = __fadd_rn(acc[2 * q], bf16_lo(w[q]));
-          acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_hi(w[q]));
+      for (int i = 0; i < kU; ++i) {
+        const int vec = vb + i * kCtaThreads;
+        if (vec >= V) continue;
+        if (kShared) {
+          const uint4 sv = ld_nc_v4(shared + t * H + (int64_t)vec * 8);
+          const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[i][2 * q] = __fadd_rn(acc[i][2 * q], bf16_lo(w[q]));
+            acc[i][2 * q + 1] = __fadd_rn(acc[i][2 * q + 1], bf16_hi(w[q]));
+          }
         }
+        uint4 o;
+        o.x = pack_bf16x2(acc[i][0], acc[i][1]);
+        o.y = pack_bf16x2(acc[i][2], acc[i][3]);
+        o.z = pack_bf16x2(acc[i][4], acc[i][5]);
+        o.w = pack_bf16x2(acc[i][6], acc[i][7]);
+        st_v4(out + t * H + (int64_t)vec * 8, o);
       }
-      uint4 o;
-      o.x = pack_bf16x2(acc[0], acc[1]);
-      o.y = pack_bf16x2(acc[2], acc[3]);
-      o.z = pack_bf16x2(acc[4], acc[5]);
-      o.w = pack_bf16x2(acc[6], acc[7]);
-      st_v4(out + t * H + (int64_t)vec * 8, o);
     }
     __syncthreads();
     buf ^= 1;
@@ -125,13 +142,14 @@ gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restri
 #ifndef MOE_BWD_THREADS
 #define MOE_BWD_THREADS 128
 #endif
-#ifndef MOE_BWD_MINB
-#define MOE_BWD_MINB 1
-#endif
 constexpr int kBwdThreads = MOE_BWD_THREADS;
 constexpr int kBwdWarps = kBwdThreads / 32;
 
-__global__ void __launch_bounds__(kBwdThreads, MOE_BWD_MINB)
+// resident CTAs per SM asked of the register allocator, per column batch
+constexpr int bwd_min_blocks(int u) { return u == 1 ? 5 : u == 2 ? 4 : 3; }
+
+template <int kU>
+__global__ void __launch_bounds__(kBwdThreads, bwd_min_blocks(kU))
 combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ y,
                    const float* __restrict__ scales, const int32_t* __restrict__ dst_row,
                    const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
@@ -139,8 +157,9 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
                    uint16_t* __restrict__ grad_y, float* __restrict__ grad_s,
                    int32_t* status) {
   pdl_begin();
-  __shared__ int32_t s_row[MOE_MAX_TOPK];
-  __shared__ float s_sc[MOE_MAX_TOPK];
+  constexpr int kKB = kKBatch / kU;  // rows per batch
+  __shared__ int32_t s_row[2][MOE_MAX_TOPK];
+  __shared__ float s_sc[2][MOE_MAX_TOPK];
   __shared__ float s_part[kBwdWarps][MOE_MAX_TOPK];
   __shared__ int32_t s_padpref[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_pad_base[MOE_MAX_EXPERTS];
@@ -150,62 +169,82 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int V = H >> 3;
-
-  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-    if (tid < K) {
+  auto fetch = [&](int64_t t, int buf) {
+    if (tid < K && t < T) {
       int r = __ldg(dst_row + t * K + tid);
       if (r != -1 && (r < 0 || (int64_t)r >= P_cap)) {
         record_error(status, MOE_ERR_BOUNDS);
         r = -1;
       }
-      s_row[tid] = r;
-      s_sc[tid] = __ldg(scales + t * K + tid);
+      s_row[buf][tid] = r;
+      s_sc[buf][tid] = __ldg(scales + t * K + tid);
     }
-    __syncthreads();
+  };
+  int buf = 0;
+  fetch(blockIdx.x, 0);
+  __syncthreads();
 
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    fetch(t + gridDim.x, buf ^ 1);
+    const int* rows = s_row[buf];
+    const float* scs = s_sc[buf];
     float dot[MOE_MAX_TOPK];
 #pragma unroll
     for (int k = 0; k < MOE_MAX_TOPK; ++k) dot[k] = 0.0f;
 
-    for (int vec = tid; vec < V; vec += kBwdThreads) {
-      const uint4 gv = ld_nc_v4(g + t * H + (int64_t)vec * 8);
-      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-      float gf[8];
+    for (int vb = tid; vb < V; vb += kBwdThreads * kU) {
+      float gf[kU][8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        gf[2 * q] = bf16_lo(gw[q]);
-        gf[2 * q + 1] = bf16_hi(gw[q]);
+      for (int i = 0; i < kU; ++i) {
+        const int vec = vb + i * kBwdThreads;
+        const uint4 gv = vec < V ? ld_nc_v4(g + t * H + (int64_t)vec * 8) : make_uint4(0, 0, 0, 0);
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          gf[i][2 * q] = bf16_lo(gw[q]);
+          gf[i][2 * q + 1] = bf16_hi(gw[q]);
+        }
       }
 #pragma unroll
-      for (int kb = 0; kb < MOE_MAX_TOPK; kb += kKBatch) {
+      for (int kb = 0; kb < MOE_MAX_TOPK; kb += kKB) {
         if (kb >= K) break;
-        uint4 yv[kKBatch];
+        uint4 yv[kKB][kU];
 #pragma unroll
-        for (int j = 0; j < kKBatch; ++j) {
+        for (int j = 0; j < kKB; ++j) {
           const int k = kb + j;
-          const int r = k < K ? s_row[k] : -1;
-          yv[j] = r >= 0 ? ld_nc_v4(y + (int64_t)r * H + (int64_t)vec * 8) : make_uint4(0, 0, 0, 0);
+          const int r = k < K ? rows[k] : -1;
+#pragma unroll
+          for (int i = 0; i < kU; ++i) {
+            const int vec = vb + i * kBwdThreads;
+            yv[j][i] = (r >= 0 && vec < V) ? ld_nc_v4(y + (int64_t)r * H + (int64_t)vec * 8)
+                                           : make_uint4(0, 0, 0, 0);
+          }
         }
 #pragma unroll
-        for (int j = 0; j < kKBatch; ++j) {
+        for (int j = 0; j < kKB; ++j) {
           const int k = kb + j;
-          const int r = k < K ? s_row[k] : -1;
+          const int r = k < K ? rows[k] : -1;
           if (r < 0) continue;
-          const float s = s_sc[k];
-          const uint32_t yw[4] = {yv[j].x, yv[j].y, yv[j].z, yv[j].w};
+          const float sk = scs[k];
           float d = dot[k];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            d = fmaf(gf[2 * q], bf16_lo(yw[q]), d);
-            d = fmaf(gf[2 * q + 1], bf16_hi(yw[q]), d);
+          for (int i = 0; i < kU; ++i) {
+            const int vec = vb + i * kBwdThreads;
+            if (vec >= V) continue;
+            const uint32_t yw[4] = {yv[j][i].x, yv[j][i].y, yv[j][i].z, yv[j][i].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              d = fmaf(gf[i][2 * q], bf16_lo(yw[q]), d);
+              d = fmaf(gf[i][2 * q + 1], bf16_hi(yw[q]), d);
+            }
+            uint4 o;
+            o.x = pack_bf16x2(__fmul_rn(sk, gf[i][0]), __fmul_rn(sk, gf[i][1]));
+            o.y = pack_bf16x2(__fmul_rn(sk, gf[i][2]), __fmul_rn(sk, gf[i][3]));
+            o.z = pack_bf16x2(__fmul_rn(sk, gf[i][4]), __fmul_rn(sk, gf[i][5]));
+            o.w = pack_bf16x2(__fmul_rn(sk, gf[i][6]), __fmul_rn(sk, gf[i][7]));
+            st_v4(grad_y + (int64_t)r * H + (int64_t)vec * 8, o);
           }
           dot[k] = d;
-          uint4 o;
-          o.x = pack_bf16x2(__fmul_rn(s, gf[0]), __fmul_rn(s, gf[1]));
-          o.y = pack_bf16x2(__fmul_rn(s, gf[2]), __fmul_rn(s, gf[3]));
-          o.z = pack_bf16x2(__fmul_rn(s, gf[4]), __fmul_rn(s, gf[5]));
-          o.w = pack_bf16x2(__fmul_rn(s, gf[6]), __fmul_rn(s, gf[7]));
-          st_v4(grad_y + (int64_t)r * H + (int64_t)vec * 8, o);
         }
       }
     }
@@ -219,14 +258,15 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
       for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
       if (lane == 0) s_part[warp][k] = d;
     }
-    __syncthreads();
+    __syncthreads();  // partial sums ready; s_row[buf ^ 1] filled
     if (tid < K) {
       float sum = 0.0f;
 #pragma unroll
       for (int w = 0; w < kBwdWarps; ++w) sum += s_part[w][tid];
-      grad_s[t * K + tid] = s_row[tid] >= 0 ? sum : 0.0f;
+      grad_s[t * K + tid] = rows[tid] >= 0 ? sum : 0.0f;
     }
-    __syncthreads();
+    __syncthreads();  // s_part and s_row[buf] free for reuse
+    buf ^= 1;
   }
 
   // ---- zero the padding rows (below P) of grad_y ----
@@ -270,21 +310,64 @@ int blocks_per_sm(F kernel, int threads, int device, int* cache) {
   return n;
 }
 
-int g_occ_comb[4][64];
-int g_occ_bwd[64];
+int g_occ_comb[12][64];
+int g_occ_bwd[4][64];
 
-template <bool kScaled, bool kShared>
-int launch_gather(int slot, const uint16_t* y, const int32_t* dst_row, const float* scales,
-                  const uint16_t* shared, int64_t T, int K, int H, int64_t P_cap, uint16_t* out,
-                  int32_t* status, cudaStream_t s) {
+// kU = columns per thread per batch: 8 / K rounded down to a power of two,
+// and no more than the row has columns for the CTA (V / threads).
+inline int gather_u(int K, int V, int threads) {
+  int u = K <= 1 ? 8 : K == 2 ? 4 : K <= 4 ? 2 : 1;
+  while (u > 1 && u * threads > V) u >>= 1;
+  return u;
+}
+
+template <bool kScaled, bool kShared, int kU>
+int launch_gather_u(int slot, const uint16_t* y, const int32_t* dst_row, const float* scales,
+                    const uint16_t* shared, int64_t T, int K, int H, int64_t P_cap,
+                    uint16_t* out, int32_t* status, cudaStream_t s) {
   const int dev = moe_host::current_device();
-  auto kern = gather_reduce_cta_kernel<kScaled, kShared>;
+  auto kern = gather_reduce_cta_kernel<kScaled, kShared, kU>;
   const int bps = blocks_per_sm(kern, kCtaThreads, dev, g_occ_comb[slot]);
   int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
   if (grid > T) grid = T;
   if (grid < 1) grid = 1;
   return moe_host::launch(kern, dim3((unsigned)grid), dim3(kCtaThreads), 0, s, y, dst_row, scales,
                           shared, T, K, H, P_cap, out, status);
+}
+
+template <bool kScaled, bool kShared>
+int launch_gather(int slot, const uint16_t* y, const int32_t* dst_row, const float* scales,
+                  const uint16_t* shared, int64_t T, int K, int H, int64_t P_cap, uint16_t* out,
+                  int32_t* status, cudaStream_t s) {
+  switch (gather_u(K, H >> 3, kCtaThreads)) {
+    case 8:
+      return launch_gather_u<kScaled, kShared, 8>(slot * 4 + 0, y, dst_row, scales, shared, T, K,
+                                                  H, P_cap, out, status, s);
+    case 4:
+      return launch_gather_u<kScaled, kShared, 4>(slot * 4 + 1, y, dst_row, scales, shared, T, K,
+                                                  H, P_cap, out, status, s);
+    case 2:
+      return launch_gather_u<kScaled, kShared, 2>(slot * 4 + 2, y, dst_row, scales, shared, T, K,
+                                                  H, P_cap, out, status, s);
+    default:
+      return launch_gather_u<kScaled, kShared, 1>(slot * 4 + 3, y, dst_row, scales, shared, T, K,
+                                                  H, P_cap, out, status, s);
+  }
+}
+
+template <int kU>
+int launch_bwd(int slot, const uint16_t* g, const uint16_t* y, const float* scales,
+               const int32_t* dst_row, const int32_t* counts, const int32_t* offsets, int E,
+               int64_t T, int K, int H, int64_t P_cap, uint16_t* grad_y, float* grad_s,
+               int32_t* status, cudaStream_t s) {
+  const int dev = moe_host::current_device();
+  auto kern = combine_bwd_kernel<kU>;
+  const int bps = blocks_per_sm(kern, kBwdThreads, dev, g_occ_bwd[slot]);
+  int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
+  const int64_t need = T + (int64_t)(kTile - 1) * E;
+  if (grid > need) grid = need;
+  return moe_host::launch(kern, dim3((unsigned)grid), dim3(kBwdThreads), 0, s, g, y, scales,
+                          dst_row, counts, offsets, E, T, K, H, P_cap, grad_y, grad_s, status);
 }
 
 int check_rows_args(const void* y, const int32_t* dst_row, int64_t T, int K, int H,
@@ -348,14 +431,22 @@ extern "C" int moe_combine_bwd(const void* grad_out, const void* y, const float*
   if (!moe_host::aligned16(grad_y)) return MOE_ERR_INVALID_ARG;
   if (P_cap < moe_padded_capacity(T, K, E)) return MOE_ERR_CAPACITY;
   if (T == 0) return MOE_OK;  // P = 0: no rows to write
-  const int dev = moe_host::current_device();
-  const int bps = blocks_per_sm(combine_bwd_kernel, kBwdThreads, dev, g_occ_bwd);
-  int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
-  const int64_t need = T + (int64_t)(kTile - 1) * E;
-  if (grid > need) grid = need;
-  return moe_host::launch(combine_bwd_kernel, dim3((unsigned)grid), dim3(kBwdThreads), 0,
-                          static_cast<cudaStream_t>(stream), static_cast<const uint16_t*>(grad_out),
-                          static_cast<const uint16_t*>(y), scales, dst_row, expert_counts,
-                          expert_offsets, E, T, K, H, P_cap, static_cast<uint16_t*>(grad_y),
-                          grad_scales, d_status);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t* go = static_cast<const uint16_t*>(grad_out);
+  const uint16_t* yy = static_cast<const uint16_t*>(y);
+  uint16_t* gy = static_cast<uint16_t*>(grad_y);
+  switch (gather_u(K, H >> 3, kBwdThreads)) {
+    case 8:
+      return launch_bwd<8>(0, go, yy, scales, dst_row, expert_counts, expert_offsets, E, T, K, H,
+                           P_cap, gy, grad_scales, d_status, s);
+    case 4:
+      return launch_bwd<4>(1, go, yy, scales, dst_row, expert_counts, expert_offsets, E, T, K, H,
+                           P_cap, gy, grad_scales, d_status, s);
+    case 2:
+      return launch_bwd<2>(2, go, yy, scales, dst_row, expert_counts, expert_offsets, E, T, K, H,
+                           P_cap, gy, grad_scales, d_status, s);
+    default:
+      return launch_bwd<1>(3, go, yy, scales, dst_row, expert_counts, expert_offsets, E, T, K, H,
+                           P_cap, gy, grad_scales, d_status, s);
+  }
 }

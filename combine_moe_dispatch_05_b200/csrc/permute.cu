@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
   __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_cnt[MOE_MAX_EXPERTS];
   __shared__ int32_t s_padpref[MOE_MAX_EXPERTS + 1];
+  constexpr int kRing = 4;  // tokens whose rows are alive at once: >= kRelLag + 2
+  __shared__ int32_t s_rows[kRing][MOE_MAX_TOPK];
 
   const int lane = threadIdx.x;
   const int S = a.stages;
@@ -213,18 +215,48 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
   };
   // Release the rows whose bulk-store group belonged to unit ur: the token's
   // slots (after its last chunk) and the padding rows issued with the unit.
+  auto ring = [&](int64_t t) { return (int)((t - t_first) & (kRing - 1)); };
   auto release_unit = [&](int64_t ur) {  // lane 0 only
     fence_acq_rel_gpu();
     if ((ur % nch) == nch - 1) {
-      const int64_t t = unit_token(ur);
-      const int64_t sa = max(s0, t * a.K), sb = min(s1, (t + 1) * a.K);
-      for (int64_t sl = sa; sl < sb; ++sl) {
-        const int32_t r = __ldg(a.dst_row + sl);
-        if (r >= 0 && (int64_t)r < a.P_cap) atomic_add_relaxed_gpu(a.tile_ready + r / kTile, 1u);
-      }
+      const int* rows = s_rows[ring(unit_token(ur))];
+      for (int j = 0; j < a.K; ++j)
+        if (rows[j] >= 0) atomic_add_relaxed_gpu(a.tile_ready + rows[j] / kTile, 1u);
     }
     release_padding(pad_lo(ur), pad_lo(ur + 1));
   };
+
+  // Row indices (and FP8 scales) of a token are fetched one token ahead into
+  // registers -- lane j holds slot j -- and published to the shared ring when
+  // the token's first unit starts, so no dependent global load sits between
+  // a landed row and its stores.  Slots outside [s0, s1) read as -1.
+  const bool sc_in_regs = a.scale_cols <= 64;
+  int nxt_r = -1;
+  float nxt_s0 = 0.0f, nxt_s1 = 0.0f, cur_s0 = 0.0f, cur_s1 = 0.0f;
+  auto prefetch = [&](int64_t t) {  // all lanes
+    nxt_r = -1;
+    if (lane < a.K) {
+      const int64_t sl = t * a.K + lane;
+      if (sl >= s0 && sl < s1) nxt_r = (int)checked_row(a, sl);
+    }
+    if (a.scale_cols > 0 && sc_in_regs) {
+      const float* xs = a.x_scales + t * a.xs_stride;
+      nxt_s0 = lane < a.scale_cols ? __ldg(xs + lane) : 0.0f;
+      nxt_s1 = lane + 32 < a.scale_cols ? __ldg(xs + lane + 32) : 0.0f;
+    }
+  };
+  auto publish = [&](int64_t t) {  // all lanes
+    if (lane < a.K) s_rows[ring(t)][lane] = nxt_r;
+    cur_s0 = nxt_s0;
+    cur_s1 = nxt_s1;
+    __syncwarp();
+  };
+  const int64_t t_last = n_units > 0 ? unit_token(n_units - 1) : -1;
+  if (n_units > 0) {
+    prefetch(t_first);
+    publish(t_first);
+    if (t_first + 1 <= t_last) prefetch(t_first + 1);
+  }
 
   int64_t issued = 0;
   if (lane == 0)
@@ -234,6 +266,11 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
   for (int64_t u = 0; u < n_units; ++u) {
     const int s = (int)(u % S);
     const uint32_t parity = (uint32_t)((u / S) & 1);
+    if (u > 0 && (u % nch) == 0) {  // first unit of a new token
+      const int64_t tn = unit_token(u);
+      publish(tn);
+      if (tn + 1 <= t_last) prefetch(tn + 1);
+    }
     // padding first: it needs no load, so it keeps the copy engine busy
     issue_padding(pad_lo(u), pad_lo(u + 1));
     int ok = 1;
@@ -245,21 +282,27 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
     }
     const int64_t t = unit_token(u);
     const int ch = (int)(u % nch);
-    const int64_t sa = max(s0, t * a.K), sb = min(s1, (t + 1) * a.K);
+    const int* rows = s_rows[ring(t)];
 
     if (ch == 0 && a.scale_cols > 0) {  // FP8 scale row, all lanes
-      for (int64_t sl = sa; sl < sb; ++sl) {
-        const int64_t r = checked_row(a, sl);
+      for (int j = 0; j < a.K; ++j) {
+        const int64_t r = rows[j];
         if (r < 0) continue;
-        for (int cc = lane; cc < a.scale_cols; cc += 32)
-          a.xp_scales[r * a.scale_cols + cc] = __ldg(a.x_scales + t * a.xs_stride + cc);
+        float* dst = a.xp_scales + r * a.scale_cols;
+        if (sc_in_regs) {
+          if (lane < a.scale_cols) dst[lane] = cur_s0;
+          if (lane + 32 < a.scale_cols) dst[lane + 32] = cur_s1;
+        } else {
+          for (int cc = lane; cc < a.scale_cols; cc += 32)
+            dst[cc] = __ldg(a.x_scales + t * a.xs_stride + cc);
+        }
       }
     }
     if (lane == 0) {
       const uint32_t len = chunk_len(a, ch);
       const uint8_t* src = stage0 + (size_t)s * a.stage_bytes;
-      for (int64_t sl = sa; sl < sb; ++sl) {
-        const int64_t r = checked_row(a, sl);
+      for (int j = 0; j < a.K; ++j) {
+        const int64_t r = rows[j];
         if (r < 0) continue;
         bulk_store_s2g(a.xp + r * a.row_bytes + (int64_t)ch * a.chunk_cap, src, len);
       }

@@ -36,6 +36,8 @@ SIGNATURES = {
                                           _vp, _vp, _i64, _vp, _vp]),
     "moe_dispatch_permute": (_int, [_vp, _int, _i64, _int, _i64, _vp, _i64, _vp, _int, _vp, _vp,
                                     _int, _vp, _vp, _i64, _vp, _vp, _vp]),
+    "moe_dispatch_permute_quant": (_int, [_vp, _i64, _int, _i64, _vp, _int, _vp, _vp, _int, _vp,
+                                          _vp, _i64, _vp, _vp, _vp]),
     "moe_combine": (_int, [_vp, _vp, _vp, _vp, _i64, _int, _int, _i64, _vp, _vp, _vp]),
     "moe_combine_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _i64, _vp,
                                _vp, _vp, _vp]),
@@ -229,6 +231,30 @@ def moe_dispatch_permute(x: torch.Tensor, L: Layout, xp: Optional[torch.Tensor] 
         _ptr(L.tile_ready) if use_counters else None, _ptr(status), _stream(stream))
     _check(rc, "moe_dispatch_permute")
     return (xp, xp_scales) if dt == DTYPE_E4M3 else xp
+
+
+def moe_dispatch_permute_quant(x: torch.Tensor, L: Layout, xp: Optional[torch.Tensor] = None,
+                               xp_scales: Optional[torch.Tensor] = None,
+                               use_counters: bool = True, status: Optional[torch.Tensor] = None,
+                               stream=None):
+    """bf16 rows -> E4M3 codes + per-128-channel scales, written straight into
+    the expert-major buffer.  Returns (xp uint8 [P_cap, H], xp_scales)."""
+    _cuda(x, "x", torch.bfloat16, contiguous=False)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    T, H = x.shape
+    if xp is None:
+        xp = torch.empty((L.P_cap, H), dtype=torch.uint8, device=x.device)
+    if xp_scales is None:
+        xp_scales = torch.empty((L.P_cap, H // 128), dtype=torch.float32, device=x.device)
+    _cuda(xp, "xp")
+    _cuda(xp_scales, "xp_scales", torch.float32)
+    rc = lib().moe_dispatch_permute_quant(
+        _ptr(x), T, H, x.stride(0), _ptr(L.dst_row), L.K, _ptr(L.expert_counts),
+        _ptr(L.expert_offsets), L.E, _ptr(xp), _ptr(xp_scales), L.P_cap,
+        _ptr(L.tile_ready) if use_counters else None, _ptr(status), _stream(stream))
+    _check(rc, "moe_dispatch_permute_quant")
+    return xp, xp_scales
 
 
 # -------------------------------------------------------------- combine --

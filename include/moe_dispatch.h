@@ -200,6 +200,29 @@ MOE_API int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H, int
                          void* stream);
 
 /*
+ * Fused quantise-on-dispatch (the FP8 dispatch of [DEP] Testing, with the
+ * codes and scales of moe_quantize_e4m3 written straight into the
+ * expert-major buffer).  Byte for byte the same as moe_quantize_e4m3
+ * followed by moe_dispatch_permute(MOE_DTYPE_E4M3), without the
+ * intermediate code buffer:
+ *   per token t and 128-channel block b: s = amax|x| / 448 (fp32; 1 if the
+ *   block is zero), q = E4M3(x / s) (fp32 division, nearest-even,
+ *   saturating); xp[dst_row[t*K+k]] = q[t], xp_scales[dst_row[t*K+k]] = s[t];
+ *   padding rows: code 0x00, scale 0.0f; rows >= P untouched.
+ * In:  x bf16 [T, H], row stride x_row_stride elements (multiple of 8),
+ *      16-byte aligned; H % 128 == 0.
+ * Out: xp uint8 [P_cap, H] (16-byte aligned); xp_scales fp32 [P_cap, H/128];
+ *      tile_ready (nullable) as in moe_dispatch_permute.
+ * Data errors: MOE_ERR_BOUNDS as in moe_dispatch_permute.
+ */
+MOE_API int moe_dispatch_permute_quant(const void* x, int64_t T, int H, int64_t x_row_stride,
+                                       const int32_t* dst_row, int K,
+                                       const int32_t* expert_counts,
+                                       const int32_t* expert_offsets, int E, void* xp,
+                                       float* xp_scales, int64_t P_cap, uint32_t* tile_ready,
+                                       int32_t* d_status, void* stream);
+
+/*
  * Combine ([ASC] function description, expert_scales, shared_expert_x):
  *   out[t] = bf16( sum_{k=0..K-1} scales[t,k] * y[dst_row[t*K+k]] + shared_x[t] )
  * computed per element in fp32: acc = 0; acc = fma(scales[t,k], y, acc) for
