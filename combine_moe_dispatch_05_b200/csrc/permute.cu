@@ -8,11 +8,11 @@
 //
 // B200 design.  The work is pure data movement, so it is written as a bulk
 // copy engine rather than as threads moving registers:
-//   * one warp per CTA; lane 0 drives the SM's bulk-copy (TMA) unit: a
-//     non-multicast cp.async.bulk global -> shared load of each token row
-//     (or 16 KiB column chunk) into an S-stage ring, completed on an
-//     mbarrier, then K cp.async.bulk shared -> global stores of the same
-//     bytes, one per destination row.  The row is read from HBM once and
+//   * one warp per CTA (2 CTAs per SM for rows over 8 KiB, else 4); lane 0
+//     drives the SM's bulk-copy (TMA) unit: a non-multicast cp.async.bulk
+//     global -> shared load of each token row (or 16 KiB column chunk) into
+//     an S-stage ring, completed on an mbarrier, then K cp.async.bulk
+//     shared -> global stores of the same bytes, one per destination row.  The row is read from HBM once and
 //     never passes through registers.
 //   * padding rows are bulk-stored from a zero-filled shared chunk.
 //   * every CTA takes an equal contiguous run of the T*K slots and an equal
@@ -39,7 +39,7 @@ namespace {
 #define MOE_PERM_REL_LAG 2
 #endif
 #ifndef MOE_PERM_CTAS_PER_SM
-#define MOE_PERM_CTAS_PER_SM 2
+#define MOE_PERM_CTAS_PER_SM 0  // 0: chosen from the row size
 #endif
 #ifndef MOE_PERM_READ_LAG
 #define MOE_PERM_READ_LAG 1
@@ -48,7 +48,13 @@ constexpr uint32_t kMaxChunk = MOE_PERM_MAX_CHUNK;  // bytes per bulk copy
 constexpr int kMaxStages = 16;
 constexpr int kRelLag = MOE_PERM_REL_LAG;          // bulk groups in flight before a release
 constexpr int kReadLag = MOE_PERM_READ_LAG;        // bulk groups still reading before a refill
-constexpr int kPermCtasPerSm = MOE_PERM_CTAS_PER_SM;
+// Copy pipelines (CTAs) per SM.  Short rows mean more per-row bookkeeping on
+// the one issuing lane (waits, fences, counter adds) per byte moved, so they
+// get more pipelines per SM to hide it; long rows get deeper rings instead.
+inline int perm_ctas_per_sm(int64_t row_bytes) {
+  if (MOE_PERM_CTAS_PER_SM > 0) return MOE_PERM_CTAS_PER_SM;
+  return row_bytes <= 8192 ? 4 : 2;
+}
 
 struct PermArgs {
   const uint8_t* x;
@@ -415,8 +421,9 @@ extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return MOE_ERR_CUDA;
-  const size_t static_smem = (3 * MOE_MAX_EXPERTS + 2) * sizeof(int32_t);
-  const size_t per_cta = (size_t)optin / kPermCtasPerSm - static_smem - 1024;
+  const size_t static_smem = (3 * MOE_MAX_EXPERTS + 2 + 4 * MOE_MAX_TOPK) * sizeof(int32_t);
+  const int ctas_per_sm = perm_ctas_per_sm(row_bytes);
+  const size_t per_cta = (size_t)optin / ctas_per_sm - static_smem - 1024;
   int stages = (int)((per_cta - a.stage_bytes - kMaxStages * 8) / a.stage_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) stages = 2;
@@ -428,7 +435,7 @@ extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
     return MOE_ERR_CUDA;
 
   const int64_t v_bound = T * K + (int64_t)(kTile - 1) * E;
-  int64_t grid = (int64_t)moe_host::sm_count(dev) * kPermCtasPerSm;
+  int64_t grid = (int64_t)moe_host::sm_count(dev) * ctas_per_sm;
   const int64_t by_work = (v_bound + 7) / 8;
   if (grid > by_work) grid = by_work;
   if (grid < 1) grid = 1;

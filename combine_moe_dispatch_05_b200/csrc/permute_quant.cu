@@ -8,7 +8,8 @@
 // byte, but x is read once and the intermediate codes never touch HBM.
 //
 // A 128-thread CTA owns a token: thread i holds 16-byte vectors i, i+128, ...
-// of the bf16 row; the 16 threads of a half-warp share one 128-channel block,
+// of the bf16 row, four at a time with all four loads issued before any
+// math; the 16 threads of a half-warp share one 128-channel block,
 // reduce its amax with shuffles, divide by s = amax/448 in fp32 and convert
 // with saturating round-to-nearest-even.  Pairs of lanes merge their 8 codes
 // into one 16-byte store per destination row.  The next token's row indices
@@ -24,6 +25,7 @@ namespace moe {
 namespace {
 
 constexpr int kQpThreads = 128;
+constexpr int kQpU = 4;  // columns per thread per batch
 
 struct QuantPermArgs {
   const uint16_t* x;
@@ -91,38 +93,51 @@ __global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPe
   for (int64_t t = blockIdx.x; t < a.T; t += gridDim.x) {
     fetch(t + gridDim.x, buf ^ 1);
     const uint16_t* xr = a.x + t * a.x_stride;
-    for (int v = tid; v < V; v += kQpThreads) {  // whole half-warps stay together: V % 16 == 0
-      const uint4 d = ld_nc_v4(xr + (int64_t)v * 8);
-      const uint32_t w[4] = {d.x, d.y, d.z, d.w};
-      float f[8];
-      float amax = 0.0f;
+    // kQpU columns per thread per batch, all loads issued before any math;
+    // a half-warp's 16 lanes share one 128-channel block in every column
+    for (int vb = tid; vb < V; vb += kQpThreads * kQpU) {  // V % 16 == 0: half-warps stay whole
+      uint4 d[kQpU];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        f[2 * q] = bf16_lo(w[q]);
-        f[2 * q + 1] = bf16_hi(w[q]);
+      for (int i = 0; i < kQpU; ++i) {
+        const int v = vb + i * kQpThreads;
+        d[i] = v < V ? ld_nc_v4(xr + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      for (int i = 0; i < kQpU; ++i) {
+        const int v = vb + i * kQpThreads;
+        if (v >= V) break;  // uniform across the half-warp
+        const uint32_t w[4] = {d[i].x, d[i].y, d[i].z, d[i].w};
+        float f[8];
+        float amax = 0.0f;
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(half_mask, amax, o, 16));
-      const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-      uint32_t c[2] = {0u, 0u};
+        for (int q = 0; q < 4; ++q) {
+          f[2 * q] = bf16_lo(w[q]);
+          f[2 * q + 1] = bf16_hi(w[q]);
+        }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 pr = make_float2(__fdiv_rn(f[2 * q], s), __fdiv_rn(f[2 * q + 1], s));
-        const uint32_t c2 = (uint32_t)__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
-        c[q >> 1] |= c2 << (16 * (q & 1));
-      }
-      // even lanes store 16 codes: their own 8 and their odd neighbour's 8
-      const uint32_t n0 = __shfl_down_sync(half_mask, c[0], 1, 16);
-      const uint32_t n1 = __shfl_down_sync(half_mask, c[1], 1, 16);
-      const int blk = v >> 4;
-      for (int k = 0; k < K; ++k) {
-        const int r = s_row[buf][k];
-        if (r < 0) continue;
-        if ((lane & 1) == 0)
-          st_v4(a.xp + (int64_t)r * H + (int64_t)v * 8, make_uint4(c[0], c[1], n0, n1));
-        if ((lane & 15) == 0) a.xp_scales[(int64_t)r * nb + blk] = s;
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)
+          amax = fmaxf(amax, __shfl_xor_sync(half_mask, amax, o, 16));
+        const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        uint32_t c[2] = {0u, 0u};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 pr = make_float2(__fdiv_rn(f[2 * q], s), __fdiv_rn(f[2 * q + 1], s));
+          const uint32_t c2 = (uint32_t)__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
+          c[q >> 1] |= c2 << (16 * (q & 1));
+        }
+        // even lanes store 16 codes: their own 8 and their odd neighbour's 8
+        const uint32_t n0 = __shfl_down_sync(half_mask, c[0], 1, 16);
+        const uint32_t n1 = __shfl_down_sync(half_mask, c[1], 1, 16);
+        const int blk = v >> 4;
+        for (int k = 0; k < K; ++k) {
+          const int r = s_row[buf][k];
+          if (r < 0) continue;
+          if ((lane & 1) == 0)
+            st_v4(a.xp + (int64_t)r * H + (int64_t)v * 8, make_uint4(c[0], c[1], n0, n1));
+          if ((lane & 15) == 0) a.xp_scales[(int64_t)r * nb + blk] = s;
+        }
       }
     }
     // thread 0 keeps its own copy of token t's rows: other threads may refill
