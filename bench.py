@@ -310,6 +310,27 @@ def run_ours(args, world, rank, local):
            "clocks": clk.summary()}
 
     if not args.no_extra and world == 1:
+        cs = torch.zeros(((P_cap + 127) // 128,), dtype=torch.int32, device=dev)
+        st2 = ops.new_status(dev)
+        # the layout call resets the counters, so it leads both variants
+        t = time_calls(torch, [
+            ("layout_permute_then_consumer",
+             lambda: (ops.moe_dispatch_layout(ids, E, R, layout=L, status=st2),
+                      ops.moe_dispatch_permute(x, L, xp=xp, status=st2),
+                      ops.moe_wait_tiles_checksum(L, xp, checksums=cs, status=st2))),
+            ("layout_permute_with_concurrent_consumer",
+             lambda: (ops.moe_dispatch_layout(ids, E, R, layout=L, status=st2),
+                      ops.moe_dispatch_permute_consume(x, L, xp=xp, checksums=cs, status=st2))),
+        ], flush, 20, stream)
+        if ops.read_status(st2) != 0:
+            raise RuntimeError(f"device status {ops.read_status(st2)} in the overlap runs")
+        res["overlap"] = {"workload": res["config"]["workload"].replace(" fwd+bwd", ""),
+                          "what": "permute + a consumer that acquires each 128-row tile and "
+                                  "reads all of it (checksum): separate launches vs one "
+                                  "cooperative launch with consumers working while the copy runs",
+                          "us": {k: round(v, 1) for k, v in t.items()},
+                          "gain": round(1 - t["layout_permute_with_concurrent_consumer"] /
+                                        t["layout_permute_then_consumer"], 3)}
         res["other_workloads"] = extra_workloads(args, dev, flush, stream)
 
     if not args.no_e2e:

@@ -97,16 +97,26 @@ __device__ __forceinline__ int64_t checked_row(const PermArgs& a, int64_t slot) 
   return r;
 }
 
-__global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
-  pdl_begin();
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
-  __shared__ int32_t s_cnt[MOE_MAX_EXPERTS];
-  __shared__ int32_t s_padpref[MOE_MAX_EXPERTS + 1];
-  constexpr int kRing = 4;  // tokens whose rows are alive at once: >= kRelLag + 2
-  __shared__ int32_t s_rows[kRing][MOE_MAX_TOPK];
+constexpr int kRing = 4;  // tokens whose rows are alive at once: >= kRelLag + 2
 
-  const int lane = threadIdx.x;
+// Shared-memory tables of one copy pipeline.
+struct PermShared {
+  int32_t off[MOE_MAX_EXPERTS + 1];
+  int32_t cnt[MOE_MAX_EXPERTS];
+  int32_t padpref[MOE_MAX_EXPERTS + 1];
+  int32_t rows[kRing][MOE_MAX_TOPK];
+};
+
+// One copy pipeline, run by one warp: share c of G of the slots and padding
+// rows.  `smem` is the ring (stages, zero chunk, mbarriers).
+__device__ __forceinline__ void permute_warp(const PermArgs& a, const int64_t c, const int64_t G,
+                                             uint8_t* smem, PermShared& sh) {
+  int32_t* s_off = sh.off;
+  int32_t* s_cnt = sh.cnt;
+  int32_t* s_padpref = sh.padpref;
+  auto& s_rows = sh.rows;
+
+  const int lane = threadIdx.x & 31;
   const int S = a.stages;
   uint8_t* stage0 = smem;
   uint8_t* zero = smem + (size_t)S * a.stage_bytes;
@@ -144,7 +154,6 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
   // ---- this CTA's share: an equal run of slots and an equal run of padding rows ----
   const int64_t TK = a.T * a.K;
   const int64_t PAD = run;
-  const int64_t G = gridDim.x, c = blockIdx.x;
   const int64_t s0 = TK * c / G, s1 = TK * (c + 1) / G;      // slots
   const int64_t q0 = PAD * c / G, q1 = PAD * (c + 1) / G;    // padding indices
 
@@ -363,16 +372,137 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
   }
 }
 
+__global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
+  pdl_begin();
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ PermShared sh;
+  permute_warp(a, blockIdx.x, gridDim.x, smem, sh);
+}
+
+// ---------------------------------------------------------------------------
+// Producer and consumers in one cooperative launch.  Warp 0 of every CTA is a
+// copy pipeline exactly as in permute_kernel; warps 1..7 form the CTA's
+// consumer group, which takes tiles j = blockIdx.x, blockIdx.x + gridDim.x, ...
+// as soon as their counters read 128: thread 0 of the group polls
+// tile_ready[j] with ld.acquire.gpu (bounded), a named barrier orders that
+// acquire before the group's reads, and the group reduces the tile to the same
+// order-independent checksum as moe_wait_tiles_checksum (an expert stand-in
+// that must see every byte of the tile).  All CTAs are resident at once
+// (cooperative launch), so a consumer never waits on a producer that cannot
+// run.
+// ---------------------------------------------------------------------------
+constexpr int kConsumerWarps = 7;
+constexpr int kConsumerThreads = 32 * kConsumerWarps;
+constexpr int kFusedThreads = 32 + kConsumerThreads;
+constexpr int kFusedCtasPerSm = 2;
+
+struct ConsumerArgs {
+  uint32_t* checksums;
+  int64_t timeout_ns;
+};
+
+__device__ __forceinline__ void consumer_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
+// sum over words w_i, i = base + 4v + q, of w_i * (2i + 1) for the 16-byte
+// vectors v = first, first + step, ... below n4
+__device__ __forceinline__ uint32_t weighted_words(const uint4* p, int64_t n4, int64_t first,
+                                                   int64_t step, uint32_t base) {
+  uint32_t acc = 0;
+#pragma unroll 8
+  for (int64_t v = first; v < n4; v += step) {
+    const uint4 w = ld_cg_v4(p + v);
+    const uint32_t i = base + 4u * (uint32_t)v;
+    acc += w.x * (2u * i + 1u) + w.y * (2u * i + 3u) + w.z * (2u * i + 5u) + w.w * (2u * i + 7u);
+  }
+  return acc;
+}
+
+__global__ void __launch_bounds__(kFusedThreads, 1)
+permute_consume_kernel(const PermArgs a, const ConsumerArgs cs) {
+  pdl_begin();
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ PermShared sh;
+  __shared__ uint32_t s_red[kConsumerWarps];
+  __shared__ int s_ok;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) {
+    permute_warp(a, blockIdx.x, gridDim.x, smem, sh);
+    return;
+  }
+  const int ct = threadIdx.x - 32;
+  const int64_t P = __ldg(a.offsets + a.E);
+  if (P < 0 || P > a.P_cap) {  // same value for every consumer thread
+    if (ct == 0) record_error(a.status, MOE_ERR_BOUNDS);
+    return;
+  }
+  const int64_t n_tiles = P / kTile;
+  const int64_t data4 = (int64_t)kTile * a.row_bytes / 16;  // row_bytes % 16 == 0
+  const int64_t scale4 = a.scale_cols > 0 ? (int64_t)kTile * a.scale_cols / 4 : 0;
+  for (int64_t j = blockIdx.x; j < n_tiles; j += gridDim.x) {
+    if (ct == 0) {
+      int ok = 0;
+      if (read_status(a.status) == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (true) {
+          if (ld_acquire_gpu(a.tile_ready + j) == (uint32_t)kTile) {
+            ok = 1;
+            break;
+          }
+          if ((int64_t)(globaltimer_ns() - t0) > cs.timeout_ns) break;
+          __nanosleep(128);
+        }
+        if (!ok) record_error(a.status, MOE_ERR_TIMEOUT);
+      }
+      s_ok = ok;
+    }
+    consumer_bar();  // orders thread 0's acquire before the group's reads
+    const int ok = s_ok;
+    uint32_t acc = 0;
+    if (ok) {
+      acc = weighted_words(reinterpret_cast<const uint4*>(a.xp + j * kTile * a.row_bytes), data4,
+                           ct, kConsumerThreads, 0u);
+      if (scale4)
+        acc += weighted_words(
+            reinterpret_cast<const uint4*>(a.xp_scales + j * kTile * a.scale_cols), scale4, ct,
+            kConsumerThreads, (uint32_t)(4 * data4));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) s_red[warp - 1] = acc;
+    consumer_bar();
+    if (ct == 0 && ok) {
+      uint32_t sum = 0;
+      for (int w = 0; w < kConsumerWarps; ++w) sum += s_red[w];
+      cs.checksums[j] = sum;
+    }
+    consumer_bar();  // s_ok and s_red are reused by the next tile
+  }
+}
+
 }  // namespace
 }  // namespace moe
 
-extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
-                                    int64_t x_row_stride, const float* x_scales,
-                                    int64_t x_scales_row_stride, const int32_t* dst_row, int K,
-                                    const int32_t* expert_counts, const int32_t* expert_offsets,
-                                    int E, void* xp, float* xp_scales, int64_t P_cap,
-                                    uint32_t* tile_ready, int32_t* d_status, void* stream) {
-  using namespace moe;
+namespace moe {
+namespace {
+
+// Host-side checks shared by the permute entry points; fills everything in
+// PermArgs but the ring depth.  Returns MOE_OK or the status to report.
+int make_perm_args(const void* x, int dtype, int64_t T, int H, int64_t x_row_stride,
+                   const float* x_scales, int64_t x_scales_row_stride, const int32_t* dst_row,
+                   int K, const int32_t* expert_counts, const int32_t* expert_offsets, int E,
+                   void* xp, float* xp_scales, int64_t P_cap, uint32_t* tile_ready,
+                   int32_t* d_status, PermArgs* out) {
   if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_E4M3) return MOE_ERR_UNSUPPORTED;
   if (T < 0 || H <= 0 || K < 1 || K > MOE_MAX_TOPK || E < 1 || E > MOE_MAX_EXPERTS)
     return MOE_ERR_INVALID_ARG;
@@ -393,9 +523,7 @@ extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
   } else if (x_scales || xp_scales) {
     return MOE_ERR_INVALID_ARG;
   }
-  if (T == 0) return MOE_OK;  // P = 0: nothing to write
-
-  PermArgs a;
+  PermArgs& a = *out;
   a.x = static_cast<const uint8_t*>(x);
   a.x_stride_bytes = x_row_stride * elem;
   a.row_bytes = row_bytes;
@@ -416,20 +544,52 @@ extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
   a.chunk_cap = (uint32_t)(row_bytes < (int64_t)kMaxChunk ? row_bytes : kMaxChunk);
   a.stage_bytes = (a.chunk_cap + 127u) / 128u * 128u;
   a.n_chunks = (int)((row_bytes + a.chunk_cap - 1) / a.chunk_cap);
+  a.stages = 0;
+  return MOE_OK;
+}
 
-  const int dev = moe_host::current_device();
-  int optin = 0;
-  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  const size_t static_smem = (3 * MOE_MAX_EXPERTS + 2 + 4 * MOE_MAX_TOPK) * sizeof(int32_t);
-  const int ctas_per_sm = perm_ctas_per_sm(row_bytes);
+// Ring depth for `ctas_per_sm` CTAs sharing an SM's shared memory; returns the
+// dynamic shared-memory bytes, or 0 if even two stages do not fit.
+size_t size_ring(PermArgs& a, int ctas_per_sm, size_t static_smem, int optin) {
   const size_t per_cta = (size_t)optin / ctas_per_sm - static_smem - 1024;
   int stages = (int)((per_cta - a.stage_bytes - kMaxStages * 8) / a.stage_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) stages = 2;
   a.stages = stages;
   const size_t dyn = (size_t)(stages + 1) * a.stage_bytes + (size_t)stages * 8;
-  if (dyn + static_smem > (size_t)optin) return MOE_ERR_UNSUPPORTED;
+  return dyn + static_smem > (size_t)optin ? 0 : dyn;
+}
+
+int optin_smem(int dev) {
+  int optin = 0;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return -1;
+  return optin;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
+                                    int64_t x_row_stride, const float* x_scales,
+                                    int64_t x_scales_row_stride, const int32_t* dst_row, int K,
+                                    const int32_t* expert_counts, const int32_t* expert_offsets,
+                                    int E, void* xp, float* xp_scales, int64_t P_cap,
+                                    uint32_t* tile_ready, int32_t* d_status, void* stream) {
+  using namespace moe;
+  PermArgs a;
+  int st = make_perm_args(x, dtype, T, H, x_row_stride, x_scales, x_scales_row_stride, dst_row,
+                          K, expert_counts, expert_offsets, E, xp, xp_scales, P_cap, tile_ready,
+                          d_status, &a);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;  // P = 0: nothing to write
+
+  const int dev = moe_host::current_device();
+  const int optin = optin_smem(dev);
+  if (optin < 0) return MOE_ERR_CUDA;
+  const int ctas_per_sm = perm_ctas_per_sm(a.row_bytes);
+  const size_t dyn = size_ring(a, ctas_per_sm, sizeof(PermShared), optin);
+  if (dyn == 0) return MOE_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)dyn) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -441,4 +601,61 @@ extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
   if (grid < 1) grid = 1;
   return moe_host::launch(permute_kernel, dim3((unsigned)grid), dim3(32), dyn,
                           static_cast<cudaStream_t>(stream), a);
+}
+
+extern "C" int moe_dispatch_permute_consume(
+    const void* x, int dtype, int64_t T, int H, int64_t x_row_stride, const float* x_scales,
+    int64_t x_scales_row_stride, const int32_t* dst_row, int K, const int32_t* expert_counts,
+    const int32_t* expert_offsets, int E, void* xp, float* xp_scales, int64_t P_cap,
+    uint32_t* tile_ready, uint32_t* checksums, int64_t timeout_ns, int32_t* d_status,
+    void* stream) {
+  using namespace moe;
+  if (!tile_ready || !checksums || timeout_ns < 0) return MOE_ERR_INVALID_ARG;
+  PermArgs a;
+  int st = make_perm_args(x, dtype, T, H, x_row_stride, x_scales, x_scales_row_stride, dst_row,
+                          K, expert_counts, expert_offsets, E, xp, xp_scales, P_cap, tile_ready,
+                          d_status, &a);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+
+  const int dev = moe_host::current_device();
+  const int optin = optin_smem(dev);
+  if (optin < 0) return MOE_ERR_CUDA;
+  const size_t static_smem = sizeof(PermShared) + 64;
+  const size_t dyn = size_ring(a, kFusedCtasPerSm, static_smem, optin);
+  if (dyn == 0) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(permute_consume_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)dyn) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // every CTA must be resident at once (consumers wait on other CTAs' rows):
+  // a cooperative launch no larger than the device can hold
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_consume_kernel,
+                                                    kFusedThreads, dyn) != cudaSuccess ||
+      per_sm < 1)
+    return MOE_ERR_UNSUPPORTED;
+  if (per_sm > kFusedCtasPerSm) per_sm = kFusedCtasPerSm;
+  int64_t grid = (int64_t)moe_host::sm_count(dev) * per_sm;
+  const int64_t v_bound = T * K + (int64_t)(kTile - 1) * E;
+  const int64_t by_work = (v_bound + 7) / 8;
+  if (grid > by_work) grid = by_work;
+  if (grid < 1) grid = 1;
+  ConsumerArgs c;
+  c.checksums = checksums;
+  c.timeout_ns = timeout_ns;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kFusedThreads);
+  cfg.dynamicSmemBytes = dyn;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, permute_consume_kernel, a, c) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
 }

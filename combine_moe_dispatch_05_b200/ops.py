@@ -36,6 +36,9 @@ SIGNATURES = {
                                           _vp, _vp, _i64, _vp, _vp]),
     "moe_dispatch_permute": (_int, [_vp, _int, _i64, _int, _i64, _vp, _i64, _vp, _int, _vp, _vp,
                                     _int, _vp, _vp, _i64, _vp, _vp, _vp]),
+    "moe_dispatch_permute_consume": (_int, [_vp, _int, _i64, _int, _i64, _vp, _i64, _vp, _int,
+                                            _vp, _vp, _int, _vp, _vp, _i64, _vp, _vp, _i64, _vp,
+                                            _vp]),
     "moe_dispatch_permute_quant": (_int, [_vp, _i64, _int, _i64, _vp, _int, _vp, _vp, _int, _vp,
                                           _vp, _i64, _vp, _vp, _vp]),
     "moe_combine": (_int, [_vp, _vp, _vp, _vp, _i64, _int, _int, _i64, _vp, _vp, _vp]),
@@ -231,6 +234,43 @@ def moe_dispatch_permute(x: torch.Tensor, L: Layout, xp: Optional[torch.Tensor] 
         _ptr(L.tile_ready) if use_counters else None, _ptr(status), _stream(stream))
     _check(rc, "moe_dispatch_permute")
     return (xp, xp_scales) if dt == DTYPE_E4M3 else xp
+
+
+def moe_dispatch_permute_consume(x: torch.Tensor, L: Layout, xp: Optional[torch.Tensor] = None,
+                                 x_scales: Optional[torch.Tensor] = None,
+                                 xp_scales: Optional[torch.Tensor] = None,
+                                 checksums: Optional[torch.Tensor] = None,
+                                 timeout_ns: int = 10**9, status: Optional[torch.Tensor] = None,
+                                 stream=None):
+    """Permute with a concurrent tile consumer in one cooperative launch.
+    Returns (xp[, xp_scales], checksums)."""
+    _cuda(x, "x", contiguous=False)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    T, H = x.shape
+    if x.dtype == torch.bfloat16:
+        dt = DTYPE_BF16
+    elif x.dtype in (torch.uint8, torch.float8_e4m3fn):
+        dt = DTYPE_E4M3
+    else:
+        raise TypeError("x must be bfloat16 or E4M3 (uint8 / float8_e4m3fn)")
+    if xp is None:
+        xp = torch.empty((L.P_cap, H), dtype=x.dtype, device=x.device)
+    xs_stride = 0
+    if dt == DTYPE_E4M3:
+        _cuda(x_scales, "x_scales", torch.float32, contiguous=False)
+        xs_stride = x_scales.stride(0)
+        if xp_scales is None:
+            xp_scales = torch.empty((L.P_cap, H // 128), dtype=torch.float32, device=x.device)
+    if checksums is None:
+        checksums = torch.zeros(max((L.P_cap + TILE - 1) // TILE, 1), dtype=torch.int32,
+                                device=x.device)
+    rc = lib().moe_dispatch_permute_consume(
+        _ptr(x), dt, T, H, x.stride(0), _ptr(x_scales), xs_stride, _ptr(L.dst_row), L.K,
+        _ptr(L.expert_counts), _ptr(L.expert_offsets), L.E, _ptr(xp), _ptr(xp_scales), L.P_cap,
+        _ptr(L.tile_ready), _ptr(checksums), timeout_ns, _ptr(status), _stream(stream))
+    _check(rc, "moe_dispatch_permute_consume")
+    return (xp, xp_scales, checksums) if dt == DTYPE_E4M3 else (xp, checksums)
 
 
 def moe_dispatch_permute_quant(x: torch.Tensor, L: Layout, xp: Optional[torch.Tensor] = None,

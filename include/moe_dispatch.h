@@ -200,6 +200,33 @@ MOE_API int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H, int
                          void* stream);
 
 /*
+ * Counter-driven overlap: moe_dispatch_permute and a consumer of its
+ * chunk-completion counters in ONE cooperative launch ([DEP]: a consumer
+ * acquires each chunk once and must then see all of it).  Every CTA runs one
+ * copy pipeline (the permute) in warp 0 and a consumer group in warps 1..7;
+ * the group takes tiles j = its CTA index, + grid, ... as soon as
+ * tile_ready[j] reads 128 with ld.acquire.gpu, while the copy pipelines are
+ * still writing other tiles, and reduces each tile to the checksum that
+ * moe_wait_tiles_checksum defines (an expert stand-in that reads every byte
+ * of the tile, scales included).  The cooperative launch keeps all CTAs
+ * resident, so no consumer waits on a producer that cannot run.
+ * Arguments: as moe_dispatch_permute, plus tile_ready (required, zeroed by
+ * the layout call), checksums uint32 [ceil(P_cap/128)] and timeout_ns, the
+ * longest wait for one tile.  A wait that runs out sets MOE_ERR_TIMEOUT and
+ * leaves that checksum unwritten; MOE_ERR_UNSUPPORTED if the device cannot
+ * hold the cooperative grid.  Results (xp, xp_scales, counters) are those of
+ * moe_dispatch_permute.
+ */
+MOE_API int moe_dispatch_permute_consume(const void* x, int dtype, int64_t T, int H,
+                                         int64_t x_row_stride, const float* x_scales,
+                                         int64_t x_scales_row_stride, const int32_t* dst_row,
+                                         int K, const int32_t* expert_counts,
+                                         const int32_t* expert_offsets, int E, void* xp,
+                                         float* xp_scales, int64_t P_cap, uint32_t* tile_ready,
+                                         uint32_t* checksums, int64_t timeout_ns,
+                                         int32_t* d_status, void* stream);
+
+/*
  * Fused quantise-on-dispatch (the FP8 dispatch of [DEP] Testing, with the
  * codes and scales of moe_quantize_e4m3 written straight into the
  * expert-major buffer).  Byte for byte the same as moe_quantize_e4m3

@@ -139,3 +139,72 @@ def test_out_of_range_ids_are_skipped_downstream():
     mag = np.einsum("tk,tkh->th", np.abs(sc.numpy().astype(np.float64)),
                     np.abs(f64(xp_ref)[rows]) * (ref.dst_row.reshape(s.T, s.K, 1) >= 0))
     assert_bf16_close(dev_u16(out), out_ref, mag, s.K + 1, "combine with an unplaced slot")
+
+
+# ---------------------------------------------- concurrent consumer (fused) ----
+def _oracle_tiles(s, ids, data, scales=None):
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    xp_ref = np.zeros((ref.P_cap, data.shape[1]), data.dtype)
+    oracle.permute_rows(data, ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    xs_ref = None
+    if scales is not None:
+        xs_ref = np.zeros((ref.P_cap, scales.shape[1]), np.float32)
+        oracle.permute_rows(scales, ref.dst_row, s.K, ref.counts, ref.offsets, xs_ref)
+    return ref, xp_ref, xs_ref, oracle.tile_checksums(xp_ref, ref.P // 128, xs_ref)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 4])
+def test_concurrent_consumer_sees_only_complete_tiles_bf16(cfg):
+    """Producer warps and consumer warps run at the same time (one cooperative
+    launch); every tile the consumers acquire must already be complete."""
+    s = W.config(cfg)
+    ids, x = W.topk_ids(s), W.tokens(s)
+    ref, xp_ref, _, cs_ref = _oracle_tiles(s, ids, W.as_u16(x))
+    for rep in range(3):
+        st = ops.new_status()
+        L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R, status=st)
+        xp, cs = ops.moe_dispatch_permute_consume(x.to(DEV), L, status=st, timeout_ns=2 * 10**9)
+        assert ops.read_status(st) == 0
+        assert np.array_equal(cs.cpu().numpy().view(np.uint32)[:ref.P // 128], cs_ref), rep
+        assert np.array_equal(dev_u16(xp)[:ref.P], xp_ref[:ref.P])
+        assert np.all(L.tile_ready.cpu().numpy()[:ref.P // 128] == 128)
+
+
+def test_concurrent_consumer_fp8_with_scales():
+    s = W.config(3).with_(T=4000, H=1024, E=48, K=6, R=4)
+    ids, codes, xs = W.topk_ids(s), W.e4m3_codes(s), W.block_scales(s)
+    ref, xp_ref, xs_ref, cs_ref = _oracle_tiles(s, ids, codes.numpy(), xs.numpy())
+    st = ops.new_status()
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R, status=st)
+    xp, xps, cs = ops.moe_dispatch_permute_consume(codes.to(DEV), L, x_scales=xs.to(DEV),
+                                                   status=st)
+    assert ops.read_status(st) == 0
+    assert np.array_equal(cs.cpu().numpy().view(np.uint32)[:ref.P // 128], cs_ref)
+    assert np.array_equal(xp.cpu().numpy()[:ref.P], xp_ref[:ref.P])
+    assert np.array_equal(xps.cpu().numpy()[:ref.P], xs_ref[:ref.P])
+
+
+def test_vectorised_reference_consumer_matches_scalar_weights():
+    """The stream-ordered consumer reads 16 bytes at a time when aligned and
+    4 bytes otherwise; both give the oracle's checksums."""
+    s = W.config(1)
+    ids, x = W.topk_ids(s), W.tokens(s)
+    ref, xp_ref, _, cs_ref = _oracle_tiles(s, ids, W.as_u16(x))
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R)
+    xp = ops.moe_dispatch_permute(x.to(DEV), L)
+    cs16 = ops.moe_wait_tiles_checksum(L, xp)
+    # a 4-byte-aligned but not 16-byte-aligned copy takes the scalar path
+    buf = torch.zeros(xp.numel() * 2 + 8, dtype=torch.uint8, device=DEV)
+    off = buf[4:4 + xp.numel() * 2]
+    off.copy_(xp.view(torch.uint8).reshape(-1))
+    row_bytes = s.H * 2
+    cs4 = torch.zeros_like(cs16)
+    st = ops.new_status()
+    rc = ops.lib().moe_wait_tiles_checksum(
+        ops._ptr(L.tile_ready), ops._ptr(L.expert_offsets), s.E, ops._ptr(off), row_bytes, None, 0,
+        L.P_cap, ops._ptr(cs4), 10**9, ops._ptr(st), ops._stream())
+    assert rc == 0
+    assert ops.read_status(st) == 0
+    n = ref.P // 128
+    assert np.array_equal(cs16.cpu().numpy().view(np.uint32)[:n], cs_ref)
+    assert np.array_equal(cs4.cpu().numpy().view(np.uint32)[:n], cs_ref)
