@@ -122,6 +122,24 @@ __device__ __forceinline__ void bulk_load_g2s(void* smem_dst, const void* gsrc, 
       : "memory");
 }
 
+// Same, with an L2 cache policy (from make_policy_evict_last) on the source.
+__device__ __forceinline__ void bulk_load_g2s_hint(void* smem_dst, const void* gsrc,
+                                                   uint32_t bytes, uint64_t* bar,
+                                                   uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_addr(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+// L2 policy that keeps the lines it touches ahead of normal traffic.
+__device__ __forceinline__ uint64_t make_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // This CTA's shared memory -> global, tracked by bulk async-groups.
 __device__ __forceinline__ void bulk_store_s2g(void* gdst, const void* smem_src, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"

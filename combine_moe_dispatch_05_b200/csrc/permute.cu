@@ -380,14 +380,197 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Tile-ordered copy pipeline, for overlap with consumers.  The token-ordered
+// pipeline above reads each x row once but fills every tile from all CTAs,
+// so tiles complete only near the end.  Here the padded rows are cut into
+// items of 16 rows (8 per tile) dealt round-robin: CTA c fills items
+// c, c + G, ... in that order, row by row (one bulk load of the source
+// token's row, one bulk store), adding 16 to the tile's counter as each item
+// lands.  Item r belongs to tile r / 8, so tiles complete roughly in index
+// order while the copy runs.  x rows are read once per slot (K times per
+// token); most of those reads hit L2.  The row -> slot maps (row_src) of the
+// next items are fetched two items ahead into registers and published to a
+// three-slot shared ring one item ahead of use.
+// ---------------------------------------------------------------------------
+constexpr int kItemRows = 16;
+constexpr int kItemsPerTile = kTile / kItemRows;
+
+struct TileShared {
+  int32_t src[3][kItemRows];
+};
+
+__device__ __forceinline__ void permute_tiles_warp(const PermArgs& a, const int32_t* row_src,
+                                                   const int64_t c, const int64_t G,
+                                                   uint8_t* smem, TileShared& sh,
+                                                   uint32_t* tile_sums) {
+  const int lane = threadIdx.x & 31;
+  const int S = a.stages;
+  uint8_t* stage0 = smem;
+  uint8_t* zero = smem + (size_t)S * a.stage_bytes;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(zero + a.stage_bytes);
+
+  const int64_t P = __ldg(a.offsets + a.E);
+  if (P < 0 || P > a.P_cap || P % kTile != 0) {
+    if (lane == 0) record_error(a.status, MOE_ERR_BOUNDS);
+    return;
+  }
+  const int64_t n_items = P / kItemRows;
+  const int64_t ni = c < n_items ? (n_items - c + G - 1) / G : 0;  // items of this CTA
+  const int nch = a.n_chunks;
+  const int64_t per_item = (int64_t)kItemRows * nch;
+  const int64_t n_units = ni * per_item;
+
+  for (uint32_t i = lane * 16; i < a.stage_bytes; i += 32 * 16)
+    *reinterpret_cast<uint4*>(zero + i) = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_shared();
+  if (lane == 0) {
+    for (int s2 = 0; s2 < S; ++s2) mbar_init(&bar[s2], 1);
+    fence_mbarrier_init();
+  }
+  auto item_row0 = [&](int64_t m) { return (c + m * G) * kItemRows; };  // first padded row
+  // row -> slot map of one item: lane l < 16 holds row l, -1 for padding
+  int32_t pre = -1;
+  auto fetch_src = [&](int64_t m) {
+    pre = -1;
+    if (lane < kItemRows && m < ni) {
+      int32_t v = __ldg(row_src + item_row0(m) + lane);
+      if (v < -1 || (int64_t)v >= a.T * a.K) {
+        record_error(a.status, MOE_ERR_BOUNDS);
+        v = -1;
+      }
+      pre = v;
+    }
+  };
+  auto publish_src = [&](int64_t m) {
+    if (lane < kItemRows) sh.src[m % 3][lane] = pre;
+  };
+  fetch_src(0);
+  publish_src(0);
+  fetch_src(1);
+  publish_src(1);
+  fetch_src(2);  // published when item 1 starts
+  __syncwarp();
+
+  auto unit_item = [&](int64_t u) { return u / per_item; };
+  auto unit_row = [&](int64_t u) { return (int)((u / nch) % kItemRows); };
+  const uint64_t x_policy = make_policy_evict_last();
+  auto issue_load = [&](int64_t u) {  // lane 0 only
+    const int s2 = (int)(u % S);
+    const int64_t m = unit_item(u);
+    const int src = sh.src[m % 3][unit_row(u)];
+    if (src < 0) {  // padding row: nothing to load; complete the phase
+      uint64_t st;
+      asm volatile("mbarrier.arrive.shared::cta.b64 %0, [%1];"
+                   : "=l"(st)
+                   : "r"(smem_addr(&bar[s2]))
+                   : "memory");
+      (void)st;
+      return;
+    }
+    const int ch = (int)(u % nch);
+    const uint32_t len = chunk_len(a, ch);
+    const uint8_t* srcp =
+        a.x + (int64_t)(src / a.K) * a.x_stride_bytes + (int64_t)ch * a.chunk_cap;
+    mbar_arrive_expect_tx(&bar[s2], len);
+    // x is read once per slot: keep it in L2 for the token's other slots
+    bulk_load_g2s_hint(stage0 + (size_t)s2 * a.stage_bytes, srcp, len, &bar[s2], x_policy);
+  };
+  // Lane 0, after the item's groups completed.  The first item of a tile also
+  // clears the tile's sum that the consumers accumulate into (nullable): the
+  // clear precedes the release, and consumers add only after acquiring the
+  // complete tile, so it lands before every add.
+  auto release_item = [&](int64_t m) {
+    const int64_t row0 = item_row0(m);
+    if (tile_sums && (row0 % kTile) == 0) tile_sums[row0 / kTile] = 0u;
+    fence_acq_rel_gpu();
+    atomic_add_relaxed_gpu(a.tile_ready + row0 / kTile, (uint32_t)kItemRows);
+  };
+
+  int64_t issued = 0;
+  if (lane == 0)
+    for (; issued < n_units && issued < S; ++issued) issue_load(issued);
+
+  int64_t u_fail = -1;
+  for (int64_t u = 0; u < n_units; ++u) {
+    const int s2 = (int)(u % S);
+    const int64_t m = unit_item(u);
+    const int i = unit_row(u);
+    const int ch = (int)(u % nch);
+    if (ch == 0 && i == 0 && m >= 1) {  // item m starts: publish m + 1, fetch m + 2
+      publish_src(m + 1);
+      fetch_src(m + 2);
+      __syncwarp();
+    }
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait_bounded(&bar[s2], (uint32_t)((u / S) & 1)) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) {
+      u_fail = u;
+      break;
+    }
+    const int src = sh.src[m % 3][i];
+    const int64_t p = item_row0(m) + i;
+    if (ch == 0 && a.scale_cols > 0) {  // FP8 scale row (or zeros), all lanes
+      float* dst = a.xp_scales + p * a.scale_cols;
+      const float* xs = src >= 0 ? a.x_scales + (int64_t)(src / a.K) * a.xs_stride : nullptr;
+      for (int cc = lane; cc < a.scale_cols; cc += 32) dst[cc] = xs ? __ldg(xs + cc) : 0.0f;
+    }
+    if (lane == 0) {
+      const uint32_t len = chunk_len(a, ch);
+      const uint8_t* from = src >= 0 ? stage0 + (size_t)s2 * a.stage_bytes : zero;
+      bulk_store_s2g(a.xp + p * a.row_bytes + (int64_t)ch * a.chunk_cap, from, len);
+      bulk_commit();
+    }
+    if (a.tile_ready) {
+      __syncwarp();  // the lanes' scale stores precede lane 0's release
+      if (lane == 0) {
+        bulk_wait_all<kRelLag>();
+        const int64_t ur = u - kRelLag;
+        if (ur >= 0 && (ur + 1) % per_item == 0) {
+          fence_proxy_async_global();
+          release_item(unit_item(ur));
+        }
+      }
+    }
+    if (lane == 0) {
+      bulk_wait_read<kReadLag>();
+      if (u >= kReadLag && issued < n_units) {
+        issue_load(issued);
+        ++issued;
+      }
+    }
+  }
+  if (u_fail >= 0) {
+    if (lane == 0) {
+      record_error(a.status, MOE_ERR_TIMEOUT);
+      bulk_wait_all<0>();
+      for (int64_t u = u_fail + 1; u < issued; ++u)
+        if (!mbar_wait_bounded(&bar[u % S], (uint32_t)((u / S) & 1))) break;
+    }
+    return;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    bulk_wait_all<0>();
+    if (a.tile_ready) {
+      fence_proxy_async_global();
+      for (int64_t ur = max((int64_t)0, n_units - kRelLag); ur < n_units; ++ur)
+        if ((ur + 1) % per_item == 0) release_item(unit_item(ur));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Producer and consumers in one cooperative launch.  Warp 0 of every CTA is a
-// copy pipeline exactly as in permute_kernel; warps 1..7 form the CTA's
-// consumer group, which takes tiles j = blockIdx.x, blockIdx.x + gridDim.x, ...
-// as soon as their counters read 128: thread 0 of the group polls
-// tile_ready[j] with ld.acquire.gpu (bounded), a named barrier orders that
-// acquire before the group's reads, and the group reduces the tile to the same
-// order-independent checksum as moe_wait_tiles_checksum (an expert stand-in
-// that must see every byte of the tile).  All CTAs are resident at once
+// tile-ordered copy pipeline (items of 16 rows, tiles completing roughly in
+// index order); warps 1..7 form the CTA's consumer group, which takes the
+// same items as its producer: for each, thread 0 of the group polls the
+// item's tile counter with ld.acquire.gpu (bounded) until the whole tile is
+// published, a named barrier orders that acquire before the group's reads,
+// and the group adds the item's share of the tile checksum defined by
+// moe_wait_tiles_checksum (weights by word position in the tile, sums mod
+// 2^32, so the order of the adds does not matter) -- an expert stand-in that
+// must see every byte.  All CTAs are resident at once
 // (cooperative launch), so a consumer never waits on a producer that cannot
 // run.
 // ---------------------------------------------------------------------------
@@ -397,6 +580,7 @@ constexpr int kFusedThreads = 32 + kConsumerThreads;
 constexpr int kFusedCtasPerSm = 2;
 
 struct ConsumerArgs {
+  const int32_t* row_src;
   uint32_t* checksums;
   int64_t timeout_ns;
 };
@@ -432,24 +616,29 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 permute_consume_kernel(const PermArgs a, const ConsumerArgs cs) {
   pdl_begin();
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ PermShared sh;
+  __shared__ TileShared sh;
   __shared__ uint32_t s_red[kConsumerWarps];
   __shared__ int s_ok;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {
-    permute_warp(a, blockIdx.x, gridDim.x, smem, sh);
+    permute_tiles_warp(a, cs.row_src, blockIdx.x, gridDim.x, smem, sh, cs.checksums);
     return;
   }
+  // consumers: the same 16-row items this CTA's producer writes, each taken
+  // once its whole tile has been published
   const int ct = threadIdx.x - 32;
   const int64_t P = __ldg(a.offsets + a.E);
-  if (P < 0 || P > a.P_cap) {  // same value for every consumer thread
+  if (P < 0 || P > a.P_cap || P % kTile != 0) {  // same value for every consumer thread
     if (ct == 0) record_error(a.status, MOE_ERR_BOUNDS);
     return;
   }
-  const int64_t n_tiles = P / kTile;
-  const int64_t data4 = (int64_t)kTile * a.row_bytes / 16;  // row_bytes % 16 == 0
-  const int64_t scale4 = a.scale_cols > 0 ? (int64_t)kTile * a.scale_cols / 4 : 0;
-  for (int64_t j = blockIdx.x; j < n_tiles; j += gridDim.x) {
+  const int64_t n_items = P / kItemRows;
+  const int64_t item4 = (int64_t)kItemRows * a.row_bytes / 16;       // 16-byte words per item
+  const int64_t tile_words = (int64_t)kTile * a.row_bytes / 4;       // data words per tile
+  const int64_t sitem4 = a.scale_cols > 0 ? (int64_t)kItemRows * a.scale_cols / 4 : 0;
+  for (int64_t r = blockIdx.x; r < n_items; r += gridDim.x) {
+    const int64_t j = r / kItemsPerTile;
+    const int q = (int)(r % kItemsPerTile);
     if (ct == 0) {
       int ok = 0;
       if (read_status(a.status) == 0) {
@@ -470,12 +659,13 @@ permute_consume_kernel(const PermArgs a, const ConsumerArgs cs) {
     const int ok = s_ok;
     uint32_t acc = 0;
     if (ok) {
-      acc = weighted_words(reinterpret_cast<const uint4*>(a.xp + j * kTile * a.row_bytes), data4,
-                           ct, kConsumerThreads, 0u);
-      if (scale4)
-        acc += weighted_words(
-            reinterpret_cast<const uint4*>(a.xp_scales + j * kTile * a.scale_cols), scale4, ct,
-            kConsumerThreads, (uint32_t)(4 * data4));
+      const int64_t row0 = r * kItemRows;
+      acc = weighted_words(reinterpret_cast<const uint4*>(a.xp + row0 * a.row_bytes), item4, ct,
+                           kConsumerThreads, (uint32_t)(q * 4 * item4));
+      if (sitem4)
+        acc += weighted_words(reinterpret_cast<const uint4*>(a.xp_scales + row0 * a.scale_cols),
+                              sitem4, ct, kConsumerThreads,
+                              (uint32_t)(tile_words + q * 4 * sitem4));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -484,9 +674,9 @@ permute_consume_kernel(const PermArgs a, const ConsumerArgs cs) {
     if (ct == 0 && ok) {
       uint32_t sum = 0;
       for (int w = 0; w < kConsumerWarps; ++w) sum += s_red[w];
-      cs.checksums[j] = sum;
+      atomicAdd(cs.checksums + j, sum);  // wraps mod 2^32: order does not matter
     }
-    consumer_bar();  // s_ok and s_red are reused by the next tile
+    consumer_bar();  // s_ok and s_red are reused by the next item
   }
 }
 
@@ -606,11 +796,13 @@ extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
 extern "C" int moe_dispatch_permute_consume(
     const void* x, int dtype, int64_t T, int H, int64_t x_row_stride, const float* x_scales,
     int64_t x_scales_row_stride, const int32_t* dst_row, int K, const int32_t* expert_counts,
-    const int32_t* expert_offsets, int E, void* xp, float* xp_scales, int64_t P_cap,
-    uint32_t* tile_ready, uint32_t* checksums, int64_t timeout_ns, int32_t* d_status,
-    void* stream) {
+    const int32_t* expert_offsets, int E, const int32_t* row_src, void* xp, float* xp_scales,
+    int64_t P_cap, uint32_t* tile_ready, uint32_t* checksums, int64_t timeout_ns,
+    int32_t* d_status, void* stream) {
   using namespace moe;
-  if (!tile_ready || !checksums || timeout_ns < 0) return MOE_ERR_INVALID_ARG;
+  if (!tile_ready || !checksums || !row_src || timeout_ns < 0) return MOE_ERR_INVALID_ARG;
+  if (xp_scales && !moe_host::aligned16(xp_scales)) return MOE_ERR_INVALID_ARG;
+  if (!moe_host::aligned4(checksums)) return MOE_ERR_INVALID_ARG;
   PermArgs a;
   int st = make_perm_args(x, dtype, T, H, x_row_stride, x_scales, x_scales_row_stride, dst_row,
                           K, expert_counts, expert_offsets, E, xp, xp_scales, P_cap, tile_ready,
@@ -621,7 +813,7 @@ extern "C" int moe_dispatch_permute_consume(
   const int dev = moe_host::current_device();
   const int optin = optin_smem(dev);
   if (optin < 0) return MOE_ERR_CUDA;
-  const size_t static_smem = sizeof(PermShared) + 64;
+  const size_t static_smem = sizeof(TileShared) + 64;
   const size_t dyn = size_ring(a, kFusedCtasPerSm, static_smem, optin);
   if (dyn == 0) return MOE_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(permute_consume_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -641,6 +833,7 @@ extern "C" int moe_dispatch_permute_consume(
   if (grid > by_work) grid = by_work;
   if (grid < 1) grid = 1;
   ConsumerArgs c;
+  c.row_src = row_src;
   c.checksums = checksums;
   c.timeout_ns = timeout_ns;
   cudaLaunchConfig_t cfg = {};

@@ -37,8 +37,8 @@ SIGNATURES = {
     "moe_dispatch_permute": (_int, [_vp, _int, _i64, _int, _i64, _vp, _i64, _vp, _int, _vp, _vp,
                                     _int, _vp, _vp, _i64, _vp, _vp, _vp]),
     "moe_dispatch_permute_consume": (_int, [_vp, _int, _i64, _int, _i64, _vp, _i64, _vp, _int,
-                                            _vp, _vp, _int, _vp, _vp, _i64, _vp, _vp, _i64, _vp,
-                                            _vp]),
+                                            _vp, _vp, _int, _vp, _vp, _vp, _i64, _vp, _vp, _i64,
+                                            _vp, _vp]),
     "moe_dispatch_permute_quant": (_int, [_vp, _i64, _int, _i64, _vp, _int, _vp, _vp, _int, _vp,
                                           _vp, _i64, _vp, _vp, _vp]),
     "moe_combine": (_int, [_vp, _vp, _vp, _vp, _i64, _int, _int, _i64, _vp, _vp, _vp]),
@@ -267,8 +267,9 @@ def moe_dispatch_permute_consume(x: torch.Tensor, L: Layout, xp: Optional[torch.
                                 device=x.device)
     rc = lib().moe_dispatch_permute_consume(
         _ptr(x), dt, T, H, x.stride(0), _ptr(x_scales), xs_stride, _ptr(L.dst_row), L.K,
-        _ptr(L.expert_counts), _ptr(L.expert_offsets), L.E, _ptr(xp), _ptr(xp_scales), L.P_cap,
-        _ptr(L.tile_ready), _ptr(checksums), timeout_ns, _ptr(status), _stream(stream))
+        _ptr(L.expert_counts), _ptr(L.expert_offsets), L.E, _ptr(L.row_src), _ptr(xp),
+        _ptr(xp_scales), L.P_cap, _ptr(L.tile_ready), _ptr(checksums), timeout_ns, _ptr(status),
+        _stream(stream))
     _check(rc, "moe_dispatch_permute_consume")
     return (xp, xp_scales, checksums) if dt == DTYPE_E4M3 else (xp, checksums)
 

@@ -200,29 +200,36 @@ MOE_API int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H, int
                          void* stream);
 
 /*
- * Counter-driven overlap: moe_dispatch_permute and a consumer of its
+ * Counter-driven overlap: the dispatch permute and a consumer of its
  * chunk-completion counters in ONE cooperative launch ([DEP]: a consumer
- * acquires each chunk once and must then see all of it).  Every CTA runs one
- * copy pipeline (the permute) in warp 0 and a consumer group in warps 1..7;
- * the group takes tiles j = its CTA index, + grid, ... as soon as
- * tile_ready[j] reads 128 with ld.acquire.gpu, while the copy pipelines are
- * still writing other tiles, and reduces each tile to the checksum that
- * moe_wait_tiles_checksum defines (an expert stand-in that reads every byte
- * of the tile, scales included).  The cooperative launch keeps all CTAs
- * resident, so no consumer waits on a producer that cannot run.
- * Arguments: as moe_dispatch_permute, plus tile_ready (required, zeroed by
- * the layout call), checksums uint32 [ceil(P_cap/128)] and timeout_ns, the
- * longest wait for one tile.  A wait that runs out sets MOE_ERR_TIMEOUT and
- * leaves that checksum unwritten; MOE_ERR_UNSUPPORTED if the device cannot
- * hold the cooperative grid.  Results (xp, xp_scales, counters) are those of
- * moe_dispatch_permute.
+ * acquires each chunk once and must then see all of it).  Warp 0 of every
+ * CTA is a tile-ordered copy pipeline: the padded rows are cut into 16-row
+ * items dealt round-robin to the CTAs, each filled row by row (source rows
+ * found through row_src) and added to its tile's counter as it lands, so
+ * tiles complete roughly in index order while the copy runs.  Warps 1..7
+ * are the CTA's consumer group: for each of the same items it waits until
+ * the item's tile counter reads 128 (ld.acquire.gpu), reads the item and
+ * adds its share of the tile's checksum, as moe_wait_tiles_checksum defines
+ * it (an expert stand-in that reads every byte, scales included; partial
+ * sums add mod 2^32, so their order does not matter).  The cooperative
+ * launch keeps all CTAs resident, so no consumer waits on a producer that
+ * cannot run.
+ * Arguments: as moe_dispatch_permute, plus row_src from the layout call
+ * (required), tile_ready (required, zeroed by the layout call), checksums
+ * uint32 [ceil(P_cap/128)] (no initialisation needed; each tile's entry is
+ * cleared before its first item is published) and timeout_ns, the longest
+ * wait for one tile; xp_scales, when given, 16-byte aligned.  A wait that
+ * runs out sets MOE_ERR_TIMEOUT (that tile's checksum is then incomplete);
+ * MOE_ERR_UNSUPPORTED if the device cannot hold the cooperative grid.  xp,
+ * xp_scales and the counters end as after moe_dispatch_permute.
  */
 MOE_API int moe_dispatch_permute_consume(const void* x, int dtype, int64_t T, int H,
                                          int64_t x_row_stride, const float* x_scales,
                                          int64_t x_scales_row_stride, const int32_t* dst_row,
                                          int K, const int32_t* expert_counts,
-                                         const int32_t* expert_offsets, int E, void* xp,
-                                         float* xp_scales, int64_t P_cap, uint32_t* tile_ready,
+                                         const int32_t* expert_offsets, int E,
+                                         const int32_t* row_src, void* xp, float* xp_scales,
+                                         int64_t P_cap, uint32_t* tile_ready,
                                          uint32_t* checksums, int64_t timeout_ns,
                                          int32_t* d_status, void* stream);
 
