@@ -332,6 +332,7 @@ def run_ours(args, world, rank, local):
                           "gain": round(1 - t["layout_permute_with_concurrent_consumer"] /
                                         t["layout_permute_then_consumer"], 3)}
         res["other_workloads"] = extra_workloads(args, dev, flush, stream)
+        res["planner"] = plan_on(L, E, R, ops)
 
     if not args.no_e2e:
         res["e2e"] = e2e(args, ops, torch, dev, stream, L, (ids_h, sc_h, x_h, g_h),
@@ -555,6 +556,22 @@ def extra_workloads(args, dev, flush, stream):
                    "us": {k: round(v, 1) for k, v in t.items()},
                    "GBps": {k: round(b[k] / (t[k] * 1e-6) / 1e9, 1) for k in t}}
     return res
+
+
+def plan_on(L, E, R, ops):
+    """Host balance planner on this step's per-expert counts (token-bound cost
+    model: beta * N dominates b * G)."""
+    counts = L.expert_counts.cpu().tolist()
+    cost = dict(a=0.0, b=5.0, b2=1.0, c=0.0, beta=1.0, mig=0.01)
+    t0 = time.perf_counter()
+    moves, before, after = ops.moe_plan_balance(counts, R, max_moves=128, **cost)
+    us = (time.perf_counter() - t0) * 1e6
+    G = sum(1 for n in counts if n > 0)
+    N = sum(counts)
+    ideal = max(cost["a"] + cost["b"] * G / R, cost["c"] + cost["beta"] * N / R)
+    return {"cost_model": cost, "moves": len(moves), "makespan_before": before,
+            "makespan_after": after, "ideal_lower_bound": ideal,
+            "ideal_over_after": round(ideal / after, 4), "host_us": round(us, 1)}
 
 
 # --------------------------------------------------------- oracle timing --

@@ -23,7 +23,8 @@ LIB = os.path.join(PKG, "libmoe_dispatch.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--cudart", "static", "-Xcompiler", "-fPIC",
-         "-Xcompiler", "-fvisibility=hidden", "-Xcompiler", "-Wall"]
+         "-Xcompiler", "-fvisibility=hidden", "-Xcompiler", "-Wall",
+         "-Xcompiler", "-ffp-contract=off"]  # host arithmetic exactly as written
 
 
 def _nvcc() -> str:
@@ -34,7 +35,7 @@ def _nvcc() -> str:
 
 
 def sources() -> list[str]:
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _stale() -> bool:

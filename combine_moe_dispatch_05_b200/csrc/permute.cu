@@ -459,12 +459,8 @@ __device__ __forceinline__ void permute_tiles_warp(const PermArgs& a, const int3
     const int64_t m = unit_item(u);
     const int src = sh.src[m % 3][unit_row(u)];
     if (src < 0) {  // padding row: nothing to load; complete the phase
-      uint64_t st;
-      asm volatile("mbarrier.arrive.shared::cta.b64 %0, [%1];"
-                   : "=l"(st)
-                   : "r"(smem_addr(&bar[s2]))
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&bar[s2]))
                    : "memory");
-      (void)st;
       return;
     }
     const int ch = (int)(u % nch);

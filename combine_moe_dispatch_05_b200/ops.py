@@ -46,6 +46,8 @@ SIGNATURES = {
                                _vp, _vp, _vp]),
     "moe_dispatch_bwd": (_int, [_vp, _vp, _i64, _int, _int, _i64, _vp, _vp, _vp]),
     "moe_quantize_e4m3": (_int, [_vp, _i64, _int, _i64, _vp, _vp, _vp, _vp]),
+    "moe_plan_balance": (_int, [_vp, _int, _int, _vp, ctypes.c_double, _int, _vp, _vp, _vp,
+                                _vp]),
     "moe_wait_tiles_checksum": (_int, [_vp, _vp, _int, _vp, _i64, _vp, _int, _i64, _vp, _i64,
                                        _vp, _vp]),
 }
@@ -394,3 +396,31 @@ def moe_wait_tiles_checksum(L: Layout, xp: torch.Tensor, xp_scales: Optional[tor
                                        timeout_ns, _ptr(status), _stream(stream))
     _check(rc, "moe_wait_tiles_checksum")
     return checksums
+
+
+# -------------------------------------------------------------- planner --
+class _Move(ctypes.Structure):
+    _fields_ = [("expert", ctypes.c_int32), ("src_rank", ctypes.c_int32),
+                ("dst_rank", ctypes.c_int32), ("tokens", ctypes.c_int32)]
+
+
+class _Cost(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_double) for n in ("a", "b", "b2", "c", "beta", "mig")]
+
+
+def moe_plan_balance(expert_counts, R: int, a=0.0, b=1.0, b2=0.0, c=0.0, beta=0.01, mig=0.0,
+                     min_gain=0.0, max_moves=256):
+    """Host planner (no GPU).  expert_counts: host sequence of E ints.
+    Returns (moves [(expert, src, dst, tokens)], makespan_before, makespan_after)."""
+    counts = (ctypes.c_int32 * len(expert_counts))(*[int(v) for v in expert_counts])
+    cost = _Cost(a, b, b2, c, beta, mig)
+    moves = (_Move * max(max_moves, 1))()
+    n = ctypes.c_int(0)
+    mb, ma = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    rc = lib().moe_plan_balance(ctypes.cast(counts, _vp), len(expert_counts), R,
+                                ctypes.cast(ctypes.pointer(cost), _vp), float(min_gain),
+                                max_moves, ctypes.cast(moves, _vp), ctypes.byref(n),
+                                ctypes.byref(mb), ctypes.byref(ma))
+    _check(rc, "moe_plan_balance")
+    out = [(m.expert, m.src_rank, m.dst_rank, m.tokens) for m in moves[:n.value]]
+    return out, mb.value, ma.value

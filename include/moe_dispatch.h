@@ -328,6 +328,40 @@ MOE_API int moe_wait_tiles_checksum(const uint32_t* tile_ready, const int32_t* e
                             int scale_cols, int64_t P_cap, uint32_t* checksums,
                             int64_t timeout_ns, int32_t* d_status, void* stream);
 
+/*
+ * Host balance planner over the layout's per-expert counts (host memory;
+ * copy expert_counts back first).  Sources: the DeepEP pull request's
+ * water-filling chunk-migration planner (expert-affinity batching, makespan
+ * guard, cost-aware no-op, 128-aligned fine-balance pass; section "Python")
+ * and TEMPO's max-affine cost (summary, section 2): a logical rank's time is
+ *   t_r = max(a + b*G + b2*(tiles - G), c + beta*N) + mig * (tokens moved in)
+ * with G the experts that have tokens on r, N its tokens and tiles the sum of
+ * their ceil(n / 128).  Rank r starts with the experts [r*E/R, (r+1)*E/R).
+ * Each step pairs the most expensive rank (src, lowest index on ties) with
+ * the cheapest (dst) and moves 128-token chunks (the remainder when fewer
+ * are left) of one expert: experts already on dst first, then most tokens
+ * on src, then lower id.  Pass 1 moves the most whole chunks that keep dst
+ * no costlier than src (at least one); pass 2 moves one chunk.  A move is
+ * kept only if it lowers the makespan by more than min_gain (>= 0); a pass
+ * ends when no candidate helps or max_moves moves exist.  Costs are double,
+ * evaluated in the order written, so plans are reproducible bit for bit.
+ * Out: moves[0..*n_moves) in the order made, makespans before and after
+ * (either pointer may be NULL).  No GPU work; returns MOE_ERR_INVALID_ARG
+ * on bad sizes (E % R != 0, E > 512, negative counts).
+ */
+typedef struct {
+  int32_t expert, src_rank, dst_rank, tokens;
+} moe_move_t;
+
+typedef struct {
+  double a, b, b2, c, beta, mig;
+} moe_cost_model_t;
+
+MOE_API int moe_plan_balance(const int32_t* expert_counts, int E, int R,
+                             const moe_cost_model_t* cost, double min_gain, int max_moves,
+                             moe_move_t* moves, int* n_moves, double* makespan_before,
+                             double* makespan_after);
+
 #ifdef __cplusplus
 }
 #endif
