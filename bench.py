@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--fwd-only", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="time each step as one CUDA graph replay (captured once)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the per-call timings of the other workloads")
     return ap.parse_args()
@@ -256,21 +258,46 @@ def run_ours(args, world, rank, local):
     P = int(L.expert_offsets[E].item())
     nbytes = step_bytes(T, K, H, E, P, args.fwd_only)
 
+    graph = None
+    if args.graph:  # one capture of the whole step; the timed steps replay it
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            step()
+        torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(smi_id(torch, dev)) as clk:
         for i in range(args.steps):
             flush.zero_()
-            step(evs[i])
+            if graph is not None:
+                evs[i][0].record(stream)
+                graph.replay()
+                evs[i][-1].record(stream)
+            else:
+                step(evs[i])
         torch.cuda.synchronize()
     barrier(world)
     per_phase = {p: [] for p in phases}
     step_ms = []
     for e in evs:
         step_ms.append(e[0].elapsed_time(e[-1]))
-        for j, p in enumerate(phases):
-            per_phase[p].append(e[j].elapsed_time(e[j + 1]))
+        if graph is None:
+            for j, p in enumerate(phases):
+                per_phase[p].append(e[j].elapsed_time(e[j + 1]))
+    if graph is not None:  # per-kernel times from one eager pass per step
+        for i in range(min(args.steps, 50)):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+        for e in evs[:min(args.steps, 50)]:
+            for j, p in enumerate(phases):
+                per_phase[p].append(e[j].elapsed_time(e[j + 1]))
     total_ms = sum(step_ms)
     total_ms_max = max_over_ranks(total_ms, world)
     ms_per_step = total_ms_max / args.steps
@@ -302,6 +329,8 @@ def run_ours(args, world, rank, local):
                                   f" {'fwd' if args.fwd_only else 'fwd+bwd'}",
                       "P": P, "P_cap": P_cap, "bytes_per_step": bytes_step,
                       "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                      "launch": "CUDA graph replay per step" if graph is not None else
+                                "eager launches (programmatic dependent launch)",
                       "parallelism": f"replicas x{world}"},
            "phases_us": {p: round(v, 2) for p, v in phase_us.items()},
            "phases_gbs": {p: round(v, 1) for p, v in phase_gbs.items()},
