@@ -85,7 +85,8 @@ def test_combine_identity_experts_returns_x_within_an_ulp():
 
 @pytest.mark.parametrize("T,H,E,K,R,shared", [
     (1, 8, 1, 1, 1, False), (3, 16, 4, 2, 2, True), (129, 24, 9, 3, 3, False),
-    (513, 520, 33, 5, 1, True), (40, 7176, 17, 16, 1, False), (1000, 64, 512, 16, 8, True)])
+    (513, 520, 33, 5, 1, True), (40, 7176, 17, 16, 1, False), (1000, 64, 512, 16, 8, True),
+    (77, 20480, 9, 1, 3, False), (300, 4096, 8, 2, 2, True), (200, 2048, 16, 3, 4, False)])
 def test_combine_parity_edge_shapes(T, H, E, K, R, shared):
     check_combine(W.Spec("edge", T, H, E, K, R, "uniform", seed=3 + T * H), shared)
 
@@ -158,7 +159,8 @@ def test_backward_parity_workloads(cfg):
 
 @pytest.mark.parametrize("T,H,E,K,R", [(1, 8, 1, 1, 1), (77, 24, 6, 3, 2), (300, 1032, 40, 16, 4),
                                        (2, 7168, 256, 8, 8), (1000, 64, 512, 16, 8),
-                                       (500, 40, 37, 3, 1), (129, 7176, 300, 2, 2)])
+                                       (500, 40, 37, 3, 1), (129, 7176, 300, 2, 2),
+                                       (60, 20480, 6, 1, 2), (400, 4096, 8, 2, 1)])
 def test_backward_parity_edge_shapes(T, H, E, K, R):
     s = W.Spec("edge", T, H, E, K, R, "uniform", seed=11 + T + H)
     check_combine_bwd(s)

@@ -208,3 +208,29 @@ def test_vectorised_reference_consumer_matches_scalar_weights():
     n = ref.P // 128
     assert np.array_equal(cs16.cpu().numpy().view(np.uint32)[:n], cs_ref)
     assert np.array_equal(cs4.cpu().numpy().view(np.uint32)[:n], cs_ref)
+
+
+@pytest.mark.parametrize("T,H,E,K,R,fp8", [(257, 20480, 12, 3, 3, False), (190, 20480, 10, 2, 5, True),
+                                          (1500, 64, 512, 16, 8, False)])
+def test_concurrent_consumer_chunked_rows_and_many_experts(T, H, E, K, R, fp8):
+    """Rows over 16 KiB (several bulk chunks per row), scales past 64 columns,
+    and a layout with many mostly-padding tiles."""
+    s = W.config(3).with_(T=T, H=H, E=E, K=K, R=R)
+    ids = W.topk_ids(s)
+    st = ops.new_status()
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R, status=st)
+    if fp8:
+        codes, xs = W.e4m3_codes(s), W.block_scales(s)
+        ref, xp_ref, xs_ref, cs_ref = _oracle_tiles(s, ids, codes.numpy(), xs.numpy())
+        xp, xps, cs = ops.moe_dispatch_permute_consume(codes.to(DEV), L, x_scales=xs.to(DEV),
+                                                       status=st)
+        assert np.array_equal(xps.cpu().numpy()[:ref.P], xs_ref[:ref.P])
+        got = xp.cpu().numpy()[:ref.P]
+    else:
+        x = W.tokens(s)
+        ref, xp_ref, _, cs_ref = _oracle_tiles(s, ids, W.as_u16(x))
+        xp, cs = ops.moe_dispatch_permute_consume(x.to(DEV), L, status=st)
+        got = dev_u16(xp)[:ref.P]
+    assert ops.read_status(st) == 0
+    assert np.array_equal(got, xp_ref[:ref.P])
+    assert np.array_equal(cs.cpu().numpy().view(np.uint32)[:ref.P // 128], cs_ref)

@@ -160,7 +160,9 @@ def run_permute_fp8(s, codes_cpu, xs_cpu):
 
 
 @pytest.mark.parametrize("T,H,E,K,R", [(2048, 7168, 256, 8, 8), (333, 384, 12, 3, 4),
-                                       (50, 128, 3, 2, 1)])
+                                       (50, 128, 3, 2, 1),
+                                       # 20 KiB rows: two bulk chunks, 160 scale columns
+                                       (300, 20480, 24, 4, 4), (64, 8320, 8, 2, 2)])
 def test_permute_fp8_parity(T, H, E, K, R):
     s = W.config(3).with_(T=T, H=H, E=E, K=K, R=R)
     L, ref, xp, xps, xp_ref, xps_ref = run_permute_fp8(s, W.e4m3_codes(s), W.block_scales(s))

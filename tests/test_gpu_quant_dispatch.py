@@ -51,7 +51,8 @@ def run(s, strided=False):
 
 @pytest.mark.parametrize("T,H,E,K,R", [(2000, 7168, 256, 8, 8), (333, 384, 12, 3, 4),
                                        (50, 128, 3, 2, 1), (1, 128, 1, 1, 1),
-                                       (700, 1152, 512, 16, 8), (129, 896, 7, 7, 7)])
+                                       (700, 1152, 512, 16, 8), (129, 896, 7, 7, 7),
+                                       (90, 20480, 16, 4, 4)])
 def test_fused_quant_dispatch_matches_oracle(T, H, E, K, R):
     run(W.config(3).with_(T=T, H=H, E=E, K=K, R=R))
 
