@@ -33,9 +33,9 @@ constexpr int kKBatch = 8;       // gathers issued before reducing
 #ifndef MOE_GATHER_CTA_THREADS
 #define MOE_GATHER_CTA_THREADS 256
 #endif
-#ifndef MOE_GATHER_MINB
-#define MOE_GATHER_MINB 1
-#endif
+// resident 256-thread CTAs per SM asked of the register allocator, per column
+// batch: 4 (64 registers) for one column, fewer as the batch holds more loads
+constexpr int gather_min_blocks(int u) { return u == 1 ? 4 : u == 2 ? 3 : u == 4 ? 2 : 1; }
 constexpr int kCtaThreads = MOE_GATHER_CTA_THREADS;
 
 // CTA-per-token reduction: threads 0..K-1 fetch the next token's row indices
@@ -45,7 +45,7 @@ constexpr int kCtaThreads = MOE_GATHER_CTA_THREADS;
 // before reducing, so about eight loads are in flight per thread whatever K
 // is (kU = 8 / K rounded down to a power of two).
 template <bool kScaled, bool kShared, int kU>
-__global__ void __launch_bounds__(kCtaThreads, MOE_GATHER_MINB)
+__global__ void __launch_bounds__(kCtaThreads, gather_min_blocks(kU))
 gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ dst_row,
                          const float* __restrict__ scales, const uint16_t* __restrict__ shared,
                          int64_t T, int K, int H, int64_t P_cap, uint16_t* __restrict__ out,

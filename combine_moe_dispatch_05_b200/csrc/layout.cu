@@ -143,12 +143,36 @@ layout_assign_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict_
 
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+  // this block's slots: their ranks and ids are fetched first, so those loads
+  // are in flight while the column sums below are formed
+  const int64_t t0 = (int64_t)b * tokens_per_block;
+  const int nt = (int)max((int64_t)0, min((int64_t)tokens_per_block, T - t0));
+  const int n_b = nt * K;
+  const int64_t s0 = t0 * K;
+  int my_rank[kItersPerWarp], my_id[kItersPerWarp];
+#pragma unroll
+  for (int it = 0; it < kItersPerWarp; ++it) {
+    const int i = tid + it * kLayoutThreads;
+    my_rank[it] = i < n_b ? slot_rank[s0 + i] : -1;
+    my_id[it] = i < n_b ? __ldg(ids + s0 + i) : 0;
+  }
+
   // 1. column sums of the per-block totals, split into ng interleaved groups
   const int ng = kLayoutThreads / E;  // >= 2 since E <= 512
   if (tid < ng * E) {
     const int e = tid % E, g = tid / E;
     int pre = 0, tot = 0;
-    for (int r = g; r < nb; r += ng) {
+    int r = g;
+    for (; r + 3 * ng < nb; r += 4 * ng) {  // four independent loads in flight
+      const int c0 = __ldg(block_counts + (int64_t)r * E + e);
+      const int c1 = __ldg(block_counts + (int64_t)(r + ng) * E + e);
+      const int c2 = __ldg(block_counts + (int64_t)(r + 2 * ng) * E + e);
+      const int c3 = __ldg(block_counts + (int64_t)(r + 3 * ng) * E + e);
+      tot += c0 + c1 + c2 + c3;
+      pre += (r < b ? c0 : 0) + (r + ng < b ? c1 : 0) + (r + 2 * ng < b ? c2 : 0) +
+             (r + 3 * ng < b ? c3 : 0);
+    }
+    for (; r < nb; r += ng) {
       const int c = __ldg(block_counts + (int64_t)r * E + e);
       tot += c;
       if (r < b) pre += c;
@@ -197,18 +221,17 @@ layout_assign_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict_
   }
 
   // 3. rows of this block's slots
-  const int64_t t0 = (int64_t)b * tokens_per_block;
-  const int nt = (int)max((int64_t)0, min((int64_t)tokens_per_block, T - t0));
-  const int n_b = nt * K;
-  const int64_t s0 = t0 * K;
-  for (int i = tid; i < n_b; i += kLayoutThreads) {
+#pragma unroll
+  for (int it = 0; it < kItersPerWarp; ++it) {
+    const int i = tid + it * kLayoutThreads;
+    if (i >= n_b) continue;
     const int64_t slot = s0 + i;
-    const int r = slot_rank[slot];
+    const int r = my_rank[it];
     if (r < 0) {
       dst_row[slot] = -1;
       continue;
     }
-    const int e = __ldg(ids + slot);
+    const int e = my_id[it];
     const int64_t row = (int64_t)s_off[e] + s_base[e] + r;
     if (row < 0 || row >= P_cap) {  // unreachable when P_cap passed the host check
       record_error(status, MOE_ERR_BOUNDS);
