@@ -299,19 +299,8 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
   }
 }
 
-// Blocks per SM for a kernel, cached per device.
-template <typename F>
-int blocks_per_sm(F kernel, int threads, int device, int* cache) {
-  if (device >= 0 && device < 64 && cache[device] > 0) return cache[device];
-  int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1)
-    n = 1;
-  if (device >= 0 && device < 64) cache[device] = n;
-  return n;
-}
-
-int g_occ_comb[12][64];
-int g_occ_bwd[4][64];
+std::atomic<int> g_occ_comb[12][moe_host::kMaxCachedDevices];
+std::atomic<int> g_occ_bwd[4][moe_host::kMaxCachedDevices];
 
 // kU = columns per thread per batch: 8 / K rounded down to a power of two,
 // and no more than the row has columns for the CTA (V / threads).
@@ -327,7 +316,7 @@ int launch_gather_u(int slot, const uint16_t* y, const int32_t* dst_row, const f
                     uint16_t* out, int32_t* status, cudaStream_t s) {
   const int dev = moe_host::current_device();
   auto kern = gather_reduce_cta_kernel<kScaled, kShared, kU>;
-  const int bps = blocks_per_sm(kern, kCtaThreads, dev, g_occ_comb[slot]);
+  const int bps = moe_host::blocks_per_sm(kern, kCtaThreads, 0, dev, g_occ_comb[slot]);
   int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
   if (grid > T) grid = T;
   if (grid < 1) grid = 1;
@@ -362,7 +351,7 @@ int launch_bwd(int slot, const uint16_t* g, const uint16_t* y, const float* scal
                int32_t* status, cudaStream_t s) {
   const int dev = moe_host::current_device();
   auto kern = combine_bwd_kernel<kU>;
-  const int bps = blocks_per_sm(kern, kBwdThreads, dev, g_occ_bwd[slot]);
+  const int bps = moe_host::blocks_per_sm(kern, kBwdThreads, 0, dev, g_occ_bwd[slot]);
   int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
   const int64_t need = T + (int64_t)(kTile - 1) * E;
   if (grid > need) grid = need;

@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 #include "moe_dispatch.h"
@@ -275,5 +276,27 @@ int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStr
              : MOE_ERR_CUDA;
 }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Resident blocks per SM of a kernel at a block size, looked up once per
+// device and cached (safe to call from several host threads).
+constexpr int kMaxCachedDevices = 64;
+template <typename F>
+int blocks_per_sm(F kernel, int threads, size_t dyn_smem, int device,
+                  std::atomic<int>* cache /* [kMaxCachedDevices] */) {
+  const bool cached = device >= 0 && device < kMaxCachedDevices;
+  if (cached) {
+    const int v = cache[device].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, dyn_smem) !=
+          cudaSuccess ||
+      n < 1) {
+    cudaGetLastError();
+    n = 1;
+  }
+  if (cached) cache[device].store(n, std::memory_order_relaxed);
+  return n;
+}
 
 }  // namespace moe_host

@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPe
   }
 }
 
-int g_occ_qp[64];
+std::atomic<int> g_occ_qp[moe_host::kMaxCachedDevices];
 
 }  // namespace
 }  // namespace moe
@@ -221,14 +221,7 @@ extern "C" int moe_dispatch_permute_quant(const void* x, int64_t T, int H, int64
   a.tile_ready = tile_ready;
   a.status = d_status;
   const int dev = moe_host::current_device();
-  int bps = (dev >= 0 && dev < 64) ? g_occ_qp[dev] : 0;
-  if (bps <= 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, permute_quant_kernel, kQpThreads, 0) !=
-            cudaSuccess ||
-        bps < 1)
-      bps = 1;
-    if (dev >= 0 && dev < 64) g_occ_qp[dev] = bps;
-  }
+  const int bps = moe_host::blocks_per_sm(permute_quant_kernel, kQpThreads, 0, dev, g_occ_qp);
   int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
   const int64_t need = T + (int64_t)(kTile - 1) * E;
   if (grid > need) grid = need;

@@ -26,7 +26,8 @@
  * Conventions for every call:
  *   - All pointers are DEVICE pointers unless stated; the caller owns every
  *     buffer; the library allocates no memory and keeps no state besides
- *     per-device launch settings.
+ *     cached per-device launch settings (and the fixed scratch array of
+ *     moe_dispatch_layout_static, part of the loaded library image).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
  *     enqueued on it; no call synchronises the host.
  *   - bf16 = IEEE bfloat16 (2 bytes), E4M3 = OCP 8-bit float E4M3 (1 byte).

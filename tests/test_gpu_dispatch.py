@@ -222,3 +222,23 @@ def test_quantize_then_dispatch_fp8_pipeline():
     P = ref.P
     assert np.array_equal(xp.cpu().numpy()[:P], xp_ref[:P])
     assert np.array_equal(xps.cpu().numpy()[:P], xps_ref[:P])
+
+
+def test_quantize_e4m3_round_trip_bound_on_gpu_codes():
+    """Codes and scales from the GPU quantiser, decoded by torch's own E4M3
+    conversion: |x - q*s| <= 2^-4 |x| where x/s is a normal E4M3 number and
+    <= 2^-10 s in the subnormal range (half a step of 3 mantissa bits)."""
+    s = W.config(3).with_(T=2048, H=7168)
+    x = W.tokens(s, device=DEV)
+    q, qs = ops.moe_quantize_e4m3(x)
+    deq = q.view(torch.float8_e4m3fn).float().view(s.T, s.H // 128, 128) * qs.unsqueeze(-1)
+    xv = x.float().view(s.T, s.H // 128, 128)
+    err = (deq - xv).abs()
+    r = xv.abs() / qs.unsqueeze(-1)
+    normal = r >= 2.0 ** -6
+    assert bool((err[normal] <= 2.0 ** -4 * xv.abs()[normal] * (1 + 1e-6)).all())
+    sub_bound = (2.0 ** -10 * qs.unsqueeze(-1) * (1 + 1e-6)).expand_as(xv)
+    assert bool((err[~normal] <= sub_bound[~normal]).all())
+    # every block's largest magnitude lands on +-448 exactly
+    top = torch.gather(q.view(s.T, s.H // 128, 128), 2, xv.abs().argmax(-1, keepdim=True))
+    assert bool(((top & 0x7F) == 0x7E).all())
