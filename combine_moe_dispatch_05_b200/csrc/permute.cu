@@ -559,7 +559,7 @@ __device__ __forceinline__ void permute_tiles_warp(const PermArgs& a, const int3
 // ---------------------------------------------------------------------------
 // Producer and consumers in one cooperative launch.  Warp 0 of every CTA is a
 // tile-ordered copy pipeline (items of 16 rows, tiles completing roughly in
-// index order); warps 1..7 form the CTA's consumer group, which takes the
+// index order); warps 1..3 form the CTA's consumer group, which takes the
 // same items as its producer: for each, thread 0 of the group polls the
 // item's tile counter with ld.acquire.gpu (bounded) until the whole tile is
 // published, a named barrier orders that acquire before the group's reads,
@@ -570,10 +570,10 @@ __device__ __forceinline__ void permute_tiles_warp(const PermArgs& a, const int3
 // (cooperative launch), so a consumer never waits on a producer that cannot
 // run.
 // ---------------------------------------------------------------------------
-constexpr int kConsumerWarps = 7;
+constexpr int kConsumerWarps = 3;
 constexpr int kConsumerThreads = 32 * kConsumerWarps;
 constexpr int kFusedThreads = 32 + kConsumerThreads;
-constexpr int kFusedCtasPerSm = 2;
+constexpr int kFusedCtasPerSm = 4;  // copy pipelines per SM (as for short rows)
 
 struct ConsumerArgs {
   const int32_t* row_src;

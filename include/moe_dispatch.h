@@ -207,7 +207,7 @@ MOE_API int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H, int
  * CTA is a tile-ordered copy pipeline: the padded rows are cut into 16-row
  * items dealt round-robin to the CTAs, each filled row by row (source rows
  * found through row_src) and added to its tile's counter as it lands, so
- * tiles complete roughly in index order while the copy runs.  Warps 1..7
+ * tiles complete roughly in index order while the copy runs.  Warps 1..3
  * are the CTA's consumer group: for each of the same items it waits until
  * the item's tile counter reads 128 (ld.acquire.gpu), reads the item and
  * adds its share of the tile's checksum, as moe_wait_tiles_checksum defines
