@@ -632,13 +632,100 @@ def oracle_step_sample(T_sample: int, fwd_only: bool):
     return dt, b, s
 
 
+def host_cpu():
+    """(threads this process may run on, CPU model name)."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return n, model
+
+
+def oracle_pass_partitioned(s, ids, sc, x, g, fwd_only, threads):
+    """One pass of the oracle over all s.T tokens with the tokens split into
+    `threads` contiguous ranges, one per host thread; the layout stays
+    serial.  The oracle's C loops run unchanged on each range (ctypes drops
+    the GIL for the call), and only the first range writes the padding rows.
+    Returns (seconds, outputs)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+
+    import oracle
+
+    K = s.K
+    cuts = [s.T * i // threads for i in range(threads + 1)]
+    parts = [(i, cuts[i], cuts[i + 1]) for i in range(threads) if cuts[i + 1] > cuts[i]]
+    with ThreadPoolExecutor(max_workers=max(len(parts), 1)) as pool:
+        def each(fn):
+            list(pool.map(lambda p: fn(*p), parts))
+
+        t0 = time.perf_counter()
+        L = oracle.layout(ids, s.E, s.R)
+        no_pad = np.diff(L.offsets).astype(np.int32)  # counts that leave no padding row
+        xp = np.zeros((L.P_cap, s.H), np.uint16)
+        out = np.empty((s.T, s.H), np.uint16)
+        each(lambda i, a, b: oracle.permute_rows(x[a:b], L.dst_row[a * K:b * K], K,
+                                                 L.counts if i == 0 else no_pad, L.offsets, xp))
+
+        def comb(i, a, b):
+            out[a:b] = oracle.combine(xp, L.dst_row[a * K:b * K], sc[a:b], None)
+        each(comb)
+        res = {"layout": L, "xp": xp, "out": out}
+        if not fwd_only:
+            gy = np.zeros_like(xp)
+            gs = np.empty((s.T, K), np.float32)
+            gx = np.empty((s.T, s.H), np.uint16)
+
+            def cbwd(i, a, b):
+                gs[a:b] = oracle.combine_bwd(g[a:b], xp, sc[a:b], L.dst_row[a * K:b * K],
+                                             L.counts if i == 0 else no_pad, L.offsets, gy)
+            each(cbwd)
+
+            def dbwd(i, a, b):
+                gx[a:b] = oracle.dispatch_bwd(gy, L.dst_row[a * K:b * K], b - a, K)
+            each(dbwd)
+            res.update(grad_y=gy, grad_scales=gs, grad_x=gx)
+        dt = time.perf_counter() - t0
+    return dt, res
+
+
+def cpu_baseline_all_cores(fwd_only):
+    """The whole workload (every token of one step) through the oracle on all
+    host threads, token-partitioned."""
+    from combine_moe_dispatch_05_b200 import workloads as W
+
+    n, model = host_cpu()
+    s = W.config(CONFIG_INDEX)
+    ids = W.topk_ids(s).numpy()
+    sc = W.topk_scales(s).numpy()
+    x = W.as_u16(W.tokens(s))
+    g = W.as_u16(W.grad_out(s))
+    dt, res = oracle_pass_partitioned(s, ids, sc, x, g, fwd_only, n)
+    b = sum(step_bytes(s.T, s.K, s.H, s.E, res["layout"].P, fwd_only).values())
+    return {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": n, "kind": "oracle",
+            "cpu_model": model, "seconds": round(dt, 3), "tokens_per_s": round(s.T / dt, 1),
+            "sample": f"all {s.T} tokens of one {'fwd' if fwd_only else 'fwd+bwd'} step, the "
+                      f"C oracle's loops run on {n} contiguous token ranges in parallel "
+                      f"(layout serial)"}
+
+
 ORACLE_SAMPLE_TOKENS = 1024
 
 
 def cpu_baseline(fwd_only):
     dt, b, s = oracle_step_sample(ORACLE_SAMPLE_TOKENS, fwd_only)
     return {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "seconds": round(dt, 3),
+            "cpu_model": host_cpu()[1], "host_threads": host_cpu()[0], "seconds": round(dt, 3),
             "tokens_per_s": round(ORACLE_SAMPLE_TOKENS / dt, 1),
             "sample": f"first {ORACLE_SAMPLE_TOKENS} of the {s.T} tokens of the same workload, "
                       f"one full {'fwd' if fwd_only else 'fwd+bwd'} pass of the single-threaded "
@@ -704,6 +791,7 @@ def main():
         res = run_ours(args, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(args.fwd_only)
+            res["cpu_baseline_all_cores"] = cpu_baseline_all_cores(args.fwd_only)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

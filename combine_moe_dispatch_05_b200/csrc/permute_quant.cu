@@ -7,16 +7,20 @@
 // TEMPO summary, section 1).  The result equals quantise-then-permute byte for
 // byte, but x is read once and the intermediate codes never touch HBM.
 //
-// A 128-thread CTA owns a token: thread i holds 16-byte vectors i, i+128, ...
-// of the bf16 row, four at a time with all four loads issued before any
-// math; the 16 threads of a half-warp share one 128-channel block,
-// reduce its amax with shuffles, divide by s = amax/448 in fp32 and convert
-// with saturating round-to-nearest-even.  Pairs of lanes merge their 8 codes
-// into one 16-byte store per destination row.  The next token's row indices
-// are prefetched into shared memory while the current one is processed.
-// Padding rows get code 0x00 and scale 0.  Each token's K rows are released
-// on the chunk-completion counters after a CTA barrier and one
-// fence.acq_rel.gpu.
+// A 128-thread CTA owns a token and works through its row in units of at
+// most 8192 channels: thread i holds 16-byte vectors i, i+128, ... of the
+// unit's bf16 slice, four at a time with all four loads issued before any
+// math; the 16 threads of a half-warp share one 128-channel block, reduce its
+// amax with shuffles, divide by s = amax/448 in fp32 and convert with
+// saturating round-to-nearest-even.  Codes and scales are staged once in
+// shared memory and thread 0 sends them to the K destination rows with bulk
+// stores (cp.async.bulk, no multicast), so the K-fold write fan-out costs the
+// SM's threads nothing.  Two stage buffers alternate; a stage is rewritten
+// only after the stores that read it have finished reading.  A token's rows
+// are released on the chunk-completion counters one unit later, once its
+// bulk group has completed.  Padding rows get code 0x00 and scale 0.  Where
+// a row's scales are not 16-byte aligned (H not a multiple of 512) the
+// scales are written with plain stores instead.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -25,7 +29,9 @@ namespace moe {
 namespace {
 
 constexpr int kQpThreads = 128;
-constexpr int kQpU = 4;  // columns per thread per batch
+constexpr int kQpU = 4;          // columns per thread per batch
+constexpr int kQpChunk = 8192;   // channels per unit (a multiple of 512)
+constexpr int kQpStages = 2;     // stage buffers per CTA
 
 struct QuantPermArgs {
   const uint16_t* x;
@@ -42,11 +48,19 @@ struct QuantPermArgs {
   int64_t P_cap;
   uint32_t* tile_ready;
   int32_t* status;
+  int chunk;          // channels per unit: H, or kQpChunk when H is larger
+  int stage_bytes;    // chunk codes + chunk/128 scales, rounded up to 16
+  int bulk_scales;    // scales go out by bulk store (H % 512 == 0, aligned base)
 };
+
+__host__ __device__ constexpr int qp_stage_bytes(int chunk) {
+  return (chunk + chunk / 32 + 15) / 16 * 16;
+}
 
 __global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPermArgs a) {
   pdl_begin();
-  __shared__ int32_t s_row[2][MOE_MAX_TOPK];
+  extern __shared__ __align__(128) uint8_t qp_stage[];
+  __shared__ int32_t s_row[4][MOE_MAX_TOPK];
   __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_cnt[MOE_MAX_EXPERTS];
   __shared__ int32_t s_pad[MOE_MAX_EXPERTS];
@@ -56,8 +70,9 @@ __global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPe
 
   const int tid = threadIdx.x, lane = tid & 31;
   const int E = a.E, K = a.K, H = a.H;
-  const int V = H >> 3;        // 16-byte bf16 vectors per row
   const int nb = H >> 7;       // 128-channel blocks per row
+  const int CH = a.chunk;
+  const int nch = (H + CH - 1) / CH;
   const unsigned half_mask = 0xFFFFu << (lane & 16);
 
   if (tid == 0) s_bad = 0;
@@ -77,84 +92,111 @@ __global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPe
     return;
   }
 
-  auto fetch = [&](int64_t t, int buf) {
+  // Row indices of a token sit in a ring of four: the slot of local token j
+  // is filled at the start of token j-1 and rewritten at the start of token
+  // j+3.  Thread 0 reads it to issue token j's stores (after each of token
+  // j's barriers) and to release its rows (after the first barrier of token
+  // j+1), both before it reaches the last barrier of token j+2.
+  auto fetch = [&](int64_t t, int slot) {
     if (tid < K && t < a.T) {
       int r = __ldg(a.dst_row + t * K + tid);
       if (r != -1 && (r < 0 || (int64_t)r >= a.P_cap)) {
         record_error(a.status, MOE_ERR_BOUNDS);
         r = -1;
       }
-      s_row[buf][tid] = r;
+      s_row[slot][tid] = r;
     }
   };
-  int buf = 0;
+  auto release_rows = [&](const int32_t* rows) {  // thread 0, after its group completed
+    fence_proxy_async_global();
+    fence_acq_rel_gpu();
+    for (int k = 0; k < K; ++k)
+      if (rows[k] >= 0) atomic_add_relaxed_gpu(a.tile_ready + rows[k] / kTile, 1u);
+  };
+
   fetch(blockIdx.x, 0);
   __syncthreads();
+  int slot = 0;
+  int64_t u = 0;  // units issued by this CTA
   for (int64_t t = blockIdx.x; t < a.T; t += gridDim.x) {
-    fetch(t + gridDim.x, buf ^ 1);
+    fetch(t + gridDim.x, (slot + 1) & 3);
+    const int32_t* rows = s_row[slot];
     const uint16_t* xr = a.x + t * a.x_stride;
-    // kQpU columns per thread per batch, all loads issued before any math;
-    // a half-warp's 16 lanes share one 128-channel block in every column
-    for (int vb = tid; vb < V; vb += kQpThreads * kQpU) {  // V % 16 == 0: half-warps stay whole
-      uint4 d[kQpU];
+    for (int c = 0; c < nch; ++c, ++u) {
+      const int c0 = c * CH;
+      const int cl = min(CH, H - c0);
+      const int Vn = cl >> 3;  // bf16 vectors in the unit, a multiple of 16
+      uint8_t* st_codes = qp_stage + (int)(u % kQpStages) * a.stage_bytes;
+      float* st_scl = reinterpret_cast<float*>(st_codes + CH);
+      const uint16_t* xc = xr + c0;
+      // a half-warp's 16 lanes share one 128-channel block in every column
+      for (int vb = tid; vb < Vn; vb += kQpThreads * kQpU) {
+        uint4 d[kQpU];
 #pragma unroll
-      for (int i = 0; i < kQpU; ++i) {
-        const int v = vb + i * kQpThreads;
-        d[i] = v < V ? ld_nc_v4(xr + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < kQpU; ++i) {
+          const int v = vb + i * kQpThreads;
+          d[i] = v < Vn ? ld_nc_v4(xc + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < kQpU; ++i) {
+          const int v = vb + i * kQpThreads;
+          if (v >= Vn) break;  // uniform across the half-warp
+          const uint32_t w[4] = {d[i].x, d[i].y, d[i].z, d[i].w};
+          float f[8];
+          float amax = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            f[2 * q] = bf16_lo(w[q]);
+            f[2 * q + 1] = bf16_hi(w[q]);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(half_mask, amax, o, 16));
+          const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+          uint32_t cw[2] = {0u, 0u};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 pr = make_float2(__fdiv_rn(f[2 * q], s), __fdiv_rn(f[2 * q + 1], s));
+            const uint32_t c2 = (uint32_t)__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
+            cw[q >> 1] |= c2 << (16 * (q & 1));
+          }
+          *reinterpret_cast<uint2*>(st_codes + v * 8) = make_uint2(cw[0], cw[1]);
+          if ((lane & 15) == 0) {
+            if (a.bulk_scales) {
+              st_scl[v >> 4] = s;
+            } else {
+              for (int k = 0; k < K; ++k)
+                if (rows[k] >= 0) a.xp_scales[(int64_t)rows[k] * nb + ((c0 + v * 8) >> 7)] = s;
+            }
+          }
+        }
       }
-#pragma unroll
-      for (int i = 0; i < kQpU; ++i) {
-        const int v = vb + i * kQpThreads;
-        if (v >= V) break;  // uniform across the half-warp
-        const uint32_t w[4] = {d[i].x, d[i].y, d[i].z, d[i].w};
-        float f[8];
-        float amax = 0.0f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          f[2 * q] = bf16_lo(w[q]);
-          f[2 * q + 1] = bf16_hi(w[q]);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1)
-          amax = fmaxf(amax, __shfl_xor_sync(half_mask, amax, o, 16));
-        const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-        uint32_t c[2] = {0u, 0u};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 pr = make_float2(__fdiv_rn(f[2 * q], s), __fdiv_rn(f[2 * q + 1], s));
-          const uint32_t c2 = (uint32_t)__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
-          c[q >> 1] |= c2 << (16 * (q & 1));
-        }
-        // even lanes store 16 codes: their own 8 and their odd neighbour's 8
-        const uint32_t n0 = __shfl_down_sync(half_mask, c[0], 1, 16);
-        const uint32_t n1 = __shfl_down_sync(half_mask, c[1], 1, 16);
-        const int blk = v >> 4;
+      fence_proxy_async_shared();  // this thread's stage writes precede the bulk reads
+      if (tid == 0) bulk_wait_read<kQpStages - 2>();  // the next unit's stage is free
+      __syncthreads();
+      if (tid == 0) {
         for (int k = 0; k < K; ++k) {
-          const int r = s_row[buf][k];
+          const int64_t r = rows[k];
           if (r < 0) continue;
-          if ((lane & 1) == 0)
-            st_v4(a.xp + (int64_t)r * H + (int64_t)v * 8, make_uint4(c[0], c[1], n0, n1));
-          if ((lane & 15) == 0) a.xp_scales[(int64_t)r * nb + blk] = s;
+          bulk_store_s2g(a.xp + r * H + c0, st_codes, (uint32_t)cl);
+          if (a.bulk_scales)
+            bulk_store_s2g(a.xp_scales + r * nb + (c0 >> 7), st_scl, (uint32_t)(cl >> 5));
+        }
+        bulk_commit();
+        if (a.tile_ready && c == 0 && u > 0) {
+          // the previous unit was the last of this CTA's previous token
+          bulk_wait_all<1>();
+          release_rows(s_row[(slot + 3) & 3]);
         }
       }
     }
-    // thread 0 keeps its own copy of token t's rows: other threads may refill
-    // s_row[buf] for a later token as soon as they pass the barrier
-    int rel[MOE_MAX_TOPK];
-    if (a.tile_ready && tid == 0) {
-#pragma unroll
-      for (int k = 0; k < MOE_MAX_TOPK; ++k) rel[k] = k < K ? s_row[buf][k] : -1;
-    }
-    __syncthreads();  // every row of token t is written (and s_row[buf ^ 1] is filled)
-    if (a.tile_ready && tid == 0) {
-      fence_acq_rel_gpu();
-#pragma unroll
-      for (int k = 0; k < MOE_MAX_TOPK; ++k)
-        if (rel[k] >= 0) atomic_add_relaxed_gpu(a.tile_ready + rel[k] / kTile, 1u);
-    }
-    buf ^= 1;
+    slot = (slot + 1) & 3;
+  }
+  if (tid == 0) {
+    bulk_wait_all<0>();  // stages stay alive until read; the last token's rows are written
+    if (a.tile_ready && u > 0) release_rows(s_row[(slot + 3) & 3]);
   }
 
   // ---- padding rows: code 0x00, scale 0 ----
@@ -220,11 +262,17 @@ extern "C" int moe_dispatch_permute_quant(const void* x, int64_t T, int H, int64
   a.P_cap = P_cap;
   a.tile_ready = tile_ready;
   a.status = d_status;
+  a.chunk = H < kQpChunk ? H : kQpChunk;
+  a.stage_bytes = qp_stage_bytes(a.chunk);
+  a.bulk_scales = (H % 512 == 0 && moe_host::aligned16(xp_scales)) ? 1 : 0;
+  const size_t dyn = (size_t)kQpStages * a.stage_bytes;
+  // occupancy at the largest stage size, so one cached figure holds for every H
+  const size_t dyn_max = (size_t)kQpStages * qp_stage_bytes(kQpChunk);
   const int dev = moe_host::current_device();
-  const int bps = moe_host::blocks_per_sm(permute_quant_kernel, kQpThreads, 0, dev, g_occ_qp);
+  const int bps = moe_host::blocks_per_sm(permute_quant_kernel, kQpThreads, dyn_max, dev, g_occ_qp);
   int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
   const int64_t need = T + (int64_t)(kTile - 1) * E;
   if (grid > need) grid = need;
-  return moe_host::launch(permute_quant_kernel, dim3((unsigned)grid), dim3(kQpThreads), 0,
+  return moe_host::launch(permute_quant_kernel, dim3((unsigned)grid), dim3(kQpThreads), dyn,
                           static_cast<cudaStream_t>(stream), a);
 }

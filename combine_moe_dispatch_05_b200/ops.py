@@ -1,8 +1,8 @@
 """Thin Python binding of the C ABI in include/moe_dispatch.h.
 
-Every function here only checks tensor types, allocates outputs when the
-caller did not pass them, and forwards raw device pointers, sizes and the
-current CUDA stream to the library.  All arithmetic runs in the CUDA kernels
+Every function here only checks tensor types and shapes, allocates outputs
+when the caller did not pass them, and forwards raw device pointers, sizes and
+the current CUDA stream to the library.  All arithmetic runs in the CUDA kernels
 of libmoe_dispatch.so; there is no fallback: if the library is missing or a
 tensor is not on a CUDA device, the call raises.
 """
@@ -97,6 +97,12 @@ def _cuda(t: torch.Tensor, name: str, dtype=None, contiguous=True):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if contiguous and not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _shape(t: torch.Tensor, name: str, shape):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     return t
 
 
@@ -222,14 +228,15 @@ def moe_dispatch_permute(x: torch.Tensor, L: Layout, xp: Optional[torch.Tensor] 
         raise TypeError("x must be bfloat16 or E4M3 (uint8 / float8_e4m3fn)")
     if xp is None:
         xp = torch.empty((L.P_cap, H), dtype=el, device=x.device)
-    _cuda(xp, "xp")
+    _shape(_cuda(xp, "xp"), "xp", (L.P_cap, H))
     xs_stride = 0
     if dt == DTYPE_E4M3:
         _cuda(x_scales, "x_scales", torch.float32, contiguous=False)
+        _shape(x_scales, "x_scales", (T, H // 128))
         xs_stride = x_scales.stride(0)
         if xp_scales is None:
             xp_scales = torch.empty((L.P_cap, H // 128), dtype=torch.float32, device=x.device)
-        _cuda(xp_scales, "xp_scales", torch.float32)
+        _shape(_cuda(xp_scales, "xp_scales", torch.float32), "xp_scales", (L.P_cap, H // 128))
     rc = lib().moe_dispatch_permute(
         _ptr(x), dt, T, H, x.stride(0), _ptr(x_scales), xs_stride, _ptr(L.dst_row), L.K,
         _ptr(L.expert_counts), _ptr(L.expert_offsets), L.E, _ptr(xp), _ptr(xp_scales), L.P_cap,
@@ -258,12 +265,15 @@ def moe_dispatch_permute_consume(x: torch.Tensor, L: Layout, xp: Optional[torch.
         raise TypeError("x must be bfloat16 or E4M3 (uint8 / float8_e4m3fn)")
     if xp is None:
         xp = torch.empty((L.P_cap, H), dtype=x.dtype, device=x.device)
+    _shape(_cuda(xp, "xp"), "xp", (L.P_cap, H))
     xs_stride = 0
     if dt == DTYPE_E4M3:
         _cuda(x_scales, "x_scales", torch.float32, contiguous=False)
+        _shape(x_scales, "x_scales", (T, H // 128))
         xs_stride = x_scales.stride(0)
         if xp_scales is None:
             xp_scales = torch.empty((L.P_cap, H // 128), dtype=torch.float32, device=x.device)
+        _shape(_cuda(xp_scales, "xp_scales", torch.float32), "xp_scales", (L.P_cap, H // 128))
     if checksums is None:
         checksums = torch.zeros(max((L.P_cap + TILE - 1) // TILE, 1), dtype=torch.int32,
                                 device=x.device)
@@ -290,8 +300,8 @@ def moe_dispatch_permute_quant(x: torch.Tensor, L: Layout, xp: Optional[torch.Te
         xp = torch.empty((L.P_cap, H), dtype=torch.uint8, device=x.device)
     if xp_scales is None:
         xp_scales = torch.empty((L.P_cap, H // 128), dtype=torch.float32, device=x.device)
-    _cuda(xp, "xp")
-    _cuda(xp_scales, "xp_scales", torch.float32)
+    _shape(_cuda(xp, "xp"), "xp", (L.P_cap, H))
+    _shape(_cuda(xp_scales, "xp_scales", torch.float32), "xp_scales", (L.P_cap, H // 128))
     rc = lib().moe_dispatch_permute_quant(
         _ptr(x), T, H, x.stride(0), _ptr(L.dst_row), L.K, _ptr(L.expert_counts),
         _ptr(L.expert_offsets), L.E, _ptr(xp), _ptr(xp_scales), L.P_cap,
@@ -314,7 +324,7 @@ def moe_combine(y: torch.Tensor, dst_row: torch.Tensor, scales: torch.Tensor,
         _cuda(shared_x, "shared_x", torch.bfloat16)
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
-    _cuda(out, "out", torch.bfloat16)
+    _shape(_cuda(out, "out", torch.bfloat16), "out", (T, H))
     rc = lib().moe_combine(_ptr(y), _ptr(dst_row), _ptr(scales), _ptr(shared_x), T, K, H,
                            y.shape[0] if P_cap is None else P_cap, _ptr(out), _ptr(status),
                            _stream(stream))
@@ -335,8 +345,8 @@ def moe_combine_bwd(grad_out: torch.Tensor, y: torch.Tensor, scales: torch.Tenso
         grad_y = torch.empty((L.P_cap, H), dtype=torch.bfloat16, device=y.device)
     if grad_scales is None:
         grad_scales = torch.empty((T, K), dtype=torch.float32, device=y.device)
-    _cuda(grad_y, "grad_y", torch.bfloat16)
-    _cuda(grad_scales, "grad_scales", torch.float32)
+    _shape(_cuda(grad_y, "grad_y", torch.bfloat16), "grad_y", (L.P_cap, H))
+    _shape(_cuda(grad_scales, "grad_scales", torch.float32), "grad_scales", (T, K))
     rc = lib().moe_combine_bwd(_ptr(grad_out), _ptr(y), _ptr(scales), _ptr(L.dst_row),
                                _ptr(L.expert_counts), _ptr(L.expert_offsets), L.E, T, K, H,
                                L.P_cap, _ptr(grad_y), _ptr(grad_scales), _ptr(status),
@@ -353,7 +363,7 @@ def moe_dispatch_bwd(grad_xp: torch.Tensor, dst_row: torch.Tensor, T: int, K: in
     H = grad_xp.shape[1]
     if grad_x is None:
         grad_x = torch.empty((T, H), dtype=torch.bfloat16, device=grad_xp.device)
-    _cuda(grad_x, "grad_x", torch.bfloat16)
+    _shape(_cuda(grad_x, "grad_x", torch.bfloat16), "grad_x", (T, H))
     rc = lib().moe_dispatch_bwd(_ptr(grad_xp), _ptr(dst_row), T, K, H,
                                 grad_xp.shape[0] if P_cap is None else P_cap, _ptr(grad_x),
                                 _ptr(status), _stream(stream))
@@ -373,8 +383,8 @@ def moe_quantize_e4m3(x: torch.Tensor, q: Optional[torch.Tensor] = None,
         q = torch.empty((T, H), dtype=torch.uint8, device=x.device)
     if q_scales is None:
         q_scales = torch.empty((T, H // 128), dtype=torch.float32, device=x.device)
-    _cuda(q, "q")
-    _cuda(q_scales, "q_scales", torch.float32)
+    _shape(_cuda(q, "q"), "q", (T, H))
+    _shape(_cuda(q_scales, "q_scales", torch.float32), "q_scales", (T, H // 128))
     rc = lib().moe_quantize_e4m3(_ptr(x), T, H, x.stride(0), _ptr(q), _ptr(q_scales),
                                  _ptr(status), _stream(stream))
     _check(rc, "moe_quantize_e4m3")

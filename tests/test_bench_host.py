@@ -1,0 +1,59 @@
+"""Host-side pieces of bench.py that need no GPU: the token-partitioned oracle
+run reported beside the single-threaded one must compute exactly what one
+unpartitioned oracle pass computes, and the algorithmic byte counts follow
+their per-call formulas."""
+import numpy as np
+import pytest
+
+import bench
+import oracle
+from combine_moe_dispatch_05_b200 import workloads as W
+
+
+def _serial(s, ids, sc, x, g):
+    L = oracle.layout(ids, s.E, s.R)
+    xp = np.zeros((L.P_cap, s.H), np.uint16)
+    oracle.permute_rows(x, L.dst_row, s.K, L.counts, L.offsets, xp)
+    out = oracle.combine(xp, L.dst_row, sc, None)
+    gy = np.zeros_like(xp)
+    gs = oracle.combine_bwd(g, xp, sc, L.dst_row, L.counts, L.offsets, gy)
+    gx = oracle.dispatch_bwd(gy, L.dst_row, s.T, s.K)
+    return dict(xp=xp, out=out, grad_y=gy, grad_scales=gs, grad_x=gx)
+
+
+@pytest.mark.parametrize("cfg,threads", [(1, 1), (1, 3), (1, 7), (4, 5)])
+def test_partitioned_oracle_pass_equals_one_pass(cfg, threads):
+    s = W.config(cfg)
+    if cfg != 1:
+        s = s.with_(T=200, H=256)
+    ids, sc = W.topk_ids(s).numpy(), W.topk_scales(s).numpy()
+    x, g = W.as_u16(W.tokens(s)), W.as_u16(W.grad_out(s))
+    ref = _serial(s, ids, sc, x, g)
+    _, res = bench.oracle_pass_partitioned(s, ids, sc, x, g, False, threads)
+    for key in ("xp", "out", "grad_y", "grad_x"):
+        assert np.array_equal(res[key], ref[key]), key
+    assert np.array_equal(res["grad_scales"].view(np.uint32), ref["grad_scales"].view(np.uint32))
+
+
+def test_partitioned_oracle_pass_more_threads_than_tokens():
+    s = W.config(1).with_(T=5)
+    ids, sc = W.topk_ids(s).numpy(), W.topk_scales(s).numpy()
+    x, g = W.as_u16(W.tokens(s)), W.as_u16(W.grad_out(s))
+    ref = _serial(s, ids, sc, x, g)
+    _, res = bench.oracle_pass_partitioned(s, ids, sc, x, g, False, 16)
+    assert np.array_equal(res["out"], ref["out"]) and np.array_equal(res["grad_x"], ref["grad_x"])
+
+
+def test_step_bytes_formulas():
+    T, K, H, E, P = 4096, 8, 7168, 256, 49152
+    b = bench.step_bytes(T, K, H, E, P)
+    assert b["permute"] == 2 * T * H + 2 * P * H
+    assert b["combine"] == 2 * T * K * H + 8 * T * K + 2 * T * H
+    assert b["combine_bwd"] == 2 * T * H + 2 * T * K * H + 2 * P * H + 12 * T * K
+    assert b["dispatch_bwd"] == 2 * T * K * H + 2 * T * H + 4 * T * K
+    assert set(bench.step_bytes(T, K, H, E, P, fwd_only=True)) == {"layout", "permute", "combine"}
+
+
+def test_host_cpu_reports_threads_and_model():
+    n, model = bench.host_cpu()
+    assert n >= 1 and isinstance(model, str) and model

@@ -20,7 +20,7 @@ def _lib():
     ensure_lib()
 
 
-def run(s, strided=False):
+def run(s, strided=False, scales_offset=0):
     ids = W.topk_ids(s)
     x = W.tokens(s)
     ref = oracle.layout(ids.numpy(), s.E, s.R)
@@ -39,7 +39,10 @@ def run(s, strided=False):
     else:
         xd = x.to(DEV)
     xp = torch.full((L.P_cap, s.H), 0xA5, dtype=torch.uint8, device=DEV)
-    xs = torch.full((L.P_cap, s.H // 128), -3.0, dtype=torch.float32, device=DEV)
+    # scales_offset > 0 moves the scale buffer off 16-byte alignment
+    flat = torch.full((L.P_cap * (s.H // 128) + scales_offset,), -3.0, dtype=torch.float32,
+                      device=DEV)
+    xs = flat[scales_offset:].view(L.P_cap, s.H // 128)
     ops.moe_dispatch_permute_quant(xd, L, xp=xp, xp_scales=xs, status=st)
     assert ops.read_status(st) == 0
     assert np.array_equal(xp.cpu().numpy(), xp_ref)
@@ -52,13 +55,21 @@ def run(s, strided=False):
 @pytest.mark.parametrize("T,H,E,K,R", [(2000, 7168, 256, 8, 8), (333, 384, 12, 3, 4),
                                        (50, 128, 3, 2, 1), (1, 128, 1, 1, 1),
                                        (700, 1152, 512, 16, 8), (129, 896, 7, 7, 7),
-                                       (90, 20480, 16, 4, 4)])
+                                       (90, 20480, 16, 4, 4), (61, 8704, 9, 3, 3),
+                                       (75, 8320, 6, 5, 2), (5000, 1024, 4, 2, 2)])
 def test_fused_quant_dispatch_matches_oracle(T, H, E, K, R):
     run(W.config(3).with_(T=T, H=H, E=E, K=K, R=R))
 
 
 def test_fused_quant_dispatch_strided_rows():
     run(W.config(3).with_(T=517, H=640, E=20, K=4, R=5), strided=True)
+
+
+@pytest.mark.parametrize("H", [1024, 8704])
+def test_fused_quant_dispatch_unaligned_scale_buffer(H):
+    """A scale buffer that is only 4-byte aligned takes the plain-store path
+    for the scales; codes and scales are unchanged."""
+    run(W.config(3).with_(T=300, H=H, E=10, K=3, R=2), scales_offset=1)
 
 
 def test_fused_equals_unfused_gpu_path_full_prefill():
@@ -70,10 +81,12 @@ def test_fused_equals_unfused_gpu_path_full_prefill():
     st = ops.new_status()
     L = ops.moe_dispatch_layout(ids, s.E, s.R, status=st)
     q, qs = ops.moe_quantize_e4m3(x, status=st)
-    xp1, xs1 = ops.moe_dispatch_permute(q, L, x_scales=qs, status=st)
+    xp1, xs1 = ops.moe_dispatch_permute(q, L, x_scales=qs, use_counters=False, status=st)
     P = int(L.expert_offsets[s.E])
     xp2, xs2 = ops.moe_dispatch_permute_quant(x, L, status=st)
     assert ops.read_status(st) == 0
+    cnt = L.tile_ready.cpu().numpy()
+    assert np.all(cnt[:P // 128] == 128) and np.all(cnt[P // 128:] == 0)
     assert torch.equal(xp1[:P], xp2[:P])
     assert torch.equal(xs1[:P].view(torch.int32), xs2[:P].view(torch.int32))
     # and sampled tokens against the oracle quantiser
