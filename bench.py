@@ -39,7 +39,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "dispatch+combine HBM GB/s and tokens/s on 1 B200; fraction of HBM peak"
 # kernels per step: layout (count + assign), permute, combine [, combine_bwd, dispatch_bwd]
-LAUNCHES_PER_STEP = {False: 6, True: 4}
+LAUNCHES_PER_STEP = {False: 6, True: 4}  # layout (2), permute, combine[, combine_bwd, dispatch_bwd]
 CONFIG_INDEX = 2
 FALLBACK_HBM_GBS = 6650.0
 
@@ -298,6 +298,21 @@ def run_ours(args, world, rank, local):
         for e in evs[:min(args.steps, 50)]:
             for j, p in enumerate(phases):
                 per_phase[p].append(e[j].elapsed_time(e[j + 1]))
+    snapshot = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the last timed step's outputs, checked against the oracle's pass in
+        # the cpu_baseline leg
+        snapshot = {"counts": L.expert_counts, "offsets": L.expert_offsets,
+                    "rank_counts": L.rank_counts, "rank_offsets": L.rank_offsets,
+                    "dst_row": L.dst_row, "row_src": L.row_src, "out": out.view(torch.int16)}
+        if not args.fwd_only:
+            snapshot.update(grad_y=gy.view(torch.int16), grad_scales=gs,
+                            grad_x=gx.view(torch.int16))
+        P_now = int(L.expert_offsets[E].item())
+        snapshot = {k: v.cpu().numpy() for k, v in snapshot.items()}
+        snapshot["xp"] = xp[:P_now].view(torch.int16).cpu().numpy()
+        if "grad_y" in snapshot:
+            snapshot["grad_y"] = snapshot["grad_y"][:P_now]
     total_ms = sum(step_ms)
     total_ms_max = max_over_ranks(total_ms, world)
     ms_per_step = total_ms_max / args.steps
@@ -337,6 +352,26 @@ def run_ours(args, world, rank, local):
            "roofline": roofline,
            "gpu_launches": LAUNCHES_PER_STEP[args.fwd_only] * args.steps,
            "clocks": clk.summary()}
+    if snapshot is not None:
+        res["_timed_outputs"] = snapshot
+    q = statistics.quantiles(step_ms, n=10) if len(step_ms) >= 2 else step_ms * 9
+    res["step_ms_distribution"] = {"median": round(statistics.median(step_ms), 5),
+                                   "p10": round(q[0], 5), "p90": round(q[-1], 5),
+                                   "note": "this rank's per-step event times, L2 flushed"}
+    if world == 1 and graph is None:
+        # the same step back to back without the flush: part of each step's
+        # inputs is still in L2 from the step before
+        warm = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+                for _ in range(min(args.steps, 100))]
+        for e in warm:
+            step(e)
+        torch.cuda.synchronize()
+        warm_ms = statistics.median(e[0].elapsed_time(e[-1]) for e in warm)
+        res["warm_l2"] = {"ms_per_step_median": round(warm_ms, 5),
+                          "value": round(bytes_step / (warm_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                          "note": "L2 not flushed between steps; not the headline value"}
+        if ops.read_status(st) != 0:
+            raise RuntimeError(f"device status {ops.read_status(st)} in the warm runs")
 
     if not args.no_extra and world == 1:
         cs = torch.zeros(((P_cap + 127) // 128,), dtype=torch.int32, device=dev)
@@ -561,29 +596,32 @@ def extra_workloads(args, dev, flush, stream):
     del x, xp, y, sh, out, L
     torch.cuda.empty_cache()
 
-    # backward under skew (hot expert in 60% of tokens)
-    s = W.config(5)
-    T, H, E, K, R = s.T, s.H, s.E, s.K, s.R
-    ids = W.topk_ids(s).to(dev)
-    L = ops.moe_dispatch_layout(ids, E, R)
-    y = W.expert_out(s, L.P_cap, device=dev)
-    g = W.grad_out(s, device=dev)
-    sc = W.topk_scales(s).to(dev)
-    gy = torch.empty_like(y)
-    gs = torch.empty((T, K), dtype=torch.float32, device=dev)
-    gx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    torch.cuda.synchronize()
-    P = int(L.expert_offsets[E])
-    t = time_calls(torch, [
-        ("layout", lambda: ops.moe_dispatch_layout(ids, E, R, layout=L)),
-        ("combine_bwd", lambda: ops.moe_combine_bwd(g, y, sc, L, grad_y=gy, grad_scales=gs)),
-        ("dispatch_bwd", lambda: ops.moe_dispatch_bwd(gy, L.dst_row, T, K, grad_x=gx)),
-    ], flush, steps, stream)
-    b = {"layout": 8 * T * K + 4 * P, "combine_bwd": 2 * T * H + 2 * T * K * H + 2 * P * H + 12 * T * K,
-         "dispatch_bwd": 2 * T * K * H + 2 * T * H + 4 * T * K}
-    res[s.name] = {"T": T, "H": H, "E": E, "K": K, "P": P,
-                   "us": {k: round(v, 1) for k, v in t.items()},
-                   "GBps": {k: round(b[k] / (t[k] * 1e-6) / 1e9, 1) for k in t}}
+    # backward under skew: the hot expert in 60% of the rows, and the stress variant with it in every row
+    for name, spec in (("bwd_skew", W.config(5)),
+                       ("bwd_skew_hot100", W.config(5).with_(hot_p=1.0))):
+        s = spec
+        T, H, E, K, R = s.T, s.H, s.E, s.K, s.R
+        ids = W.topk_ids(s).to(dev)
+        L = ops.moe_dispatch_layout(ids, E, R)
+        y = W.expert_out(s, L.P_cap, device=dev)
+        g = W.grad_out(s, device=dev)
+        sc = W.topk_scales(s).to(dev)
+        gy = torch.empty_like(y)
+        gs = torch.empty((T, K), dtype=torch.float32, device=dev)
+        gx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+        P = int(L.expert_offsets[E])
+        t = time_calls(torch, [
+            ("layout", lambda: ops.moe_dispatch_layout(ids, E, R, layout=L)),
+            ("combine_bwd", lambda: ops.moe_combine_bwd(g, y, sc, L, grad_y=gy, grad_scales=gs)),
+            ("dispatch_bwd", lambda: ops.moe_dispatch_bwd(gy, L.dst_row, T, K, grad_x=gx)),
+        ], flush, steps, stream)
+        b = {"layout": 8 * T * K + 4 * P,
+             "combine_bwd": 2 * T * H + 2 * T * K * H + 2 * P * H + 12 * T * K,
+             "dispatch_bwd": 2 * T * K * H + 2 * T * H + 4 * T * K}
+        res[name] = {"T": T, "H": H, "E": E, "K": K, "P": P, "hot_p": s.hot_p,
+                     "us": {k: round(v, 1) for k, v in t.items()},
+                     "GBps": {k: round(b[k] / (t[k] * 1e-6) / 1e9, 1) for k in t}}
     return res
 
 
@@ -699,9 +737,62 @@ def oracle_pass_partitioned(s, ids, sc, x, g, fwd_only, threads):
     return dt, res
 
 
-def cpu_baseline_all_cores(fwd_only):
+def bf16_max_ulp(gpu_bits, ref_bits):
+    """Largest |gpu - ref| over all elements, in units of one bf16 ulp of ref
+    (ulp of a normal r = 2^(floor(log2|r|) - 7); of zero, the smallest
+    subnormal)."""
+    import numpy as np
+
+    def f(b):
+        return (np.asarray(b).view(np.uint16).astype(np.uint32) << 16).view(np.float32) \
+            .astype(np.float64)
+    g, r = f(gpu_bits), f(ref_bits)
+    a = np.abs(r)
+    ulp = np.where(a > 0, np.exp2(np.floor(np.log2(np.where(a > 0, a, 1.0))) - 7), 2.0 ** -133)
+    return float(np.max(np.abs(g - r) / ulp)) if g.size else 0.0
+
+
+def check_timed_outputs(s, res, gpu, x, g, fwd_only):
+    """The last timed GPU step against the oracle's pass over the same inputs:
+    integers and the permuted bytes must be identical; the bf16 outputs are
+    reported as their largest error in bf16 ulps, grad_scales as its largest
+    error relative to |g_t|*|y_row| (which bounds the sum of |terms|)."""
+    import numpy as np
+
+    L = res["layout"]
+    K = s.K
+    chk = {"layout_bit_exact": bool(
+        np.array_equal(gpu["counts"], L.counts) and np.array_equal(gpu["offsets"], L.offsets)
+        and np.array_equal(gpu["dst_row"][:s.T * K], L.dst_row)
+        and np.array_equal(gpu["row_src"][:L.P_cap], L.row_src[:L.P_cap])
+        and np.array_equal(gpu["rank_counts"], L.rank_counts)
+        and np.array_equal(gpu["rank_offsets"], L.rank_offsets))}
+    P = L.P
+    chk["permute_bytes_exact"] = bool(gpu["xp"].shape[0] == P and np.array_equal(
+        gpu["xp"].view(np.uint16), res["xp"][:P]))
+    chk["combine_max_ulp"] = round(bf16_max_ulp(gpu["out"], res["out"]), 3)
+    if not fwd_only:
+        chk["combine_bwd_grad_y_max_ulp"] = round(
+            bf16_max_ulp(gpu["grad_y"], res["grad_y"][:P]), 3)
+        chk["dispatch_bwd_max_ulp"] = round(bf16_max_ulp(gpu["grad_x"], res["grad_x"]), 3)
+
+        def f(b):
+            return (b.view(np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        gn = np.linalg.norm(f(g), axis=1)                        # [T]
+        yn = np.linalg.norm(f(res["xp"]), axis=1)                # [P_cap]
+        rows = L.dst_row.reshape(s.T, K)
+        scale = np.maximum(gn[:, None] * yn[rows], 1e-30)
+        err = np.abs(gpu["grad_scales"].astype(np.float64) - res["grad_scales"].astype(np.float64))
+        chk["grad_scales_max_err_over_norms"] = float(np.max(err / scale))
+    chk["what"] = ("outputs of the last timed step against the oracle's pass over the same "
+                   "inputs (identity experts)")
+    return chk
+
+
+def cpu_baseline_all_cores(fwd_only, timed_outputs=None):
     """The whole workload (every token of one step) through the oracle on all
-    host threads, token-partitioned."""
+    host threads, token-partitioned.  Returns (baseline, check of the timed
+    GPU outputs against this pass, or None)."""
     from combine_moe_dispatch_05_b200 import workloads as W
 
     n, model = host_cpu()
@@ -712,11 +803,14 @@ def cpu_baseline_all_cores(fwd_only):
     g = W.as_u16(W.grad_out(s))
     dt, res = oracle_pass_partitioned(s, ids, sc, x, g, fwd_only, n)
     b = sum(step_bytes(s.T, s.K, s.H, s.E, res["layout"].P, fwd_only).values())
-    return {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": n, "kind": "oracle",
+    base = {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": n, "kind": "oracle",
             "cpu_model": model, "seconds": round(dt, 3), "tokens_per_s": round(s.T / dt, 1),
             "sample": f"all {s.T} tokens of one {'fwd' if fwd_only else 'fwd+bwd'} step, the "
                       f"C oracle's loops run on {n} contiguous token ranges in parallel "
                       f"(layout serial)"}
+    chk = None if timed_outputs is None else check_timed_outputs(s, res, timed_outputs, x, g,
+                                                                  fwd_only)
+    return base, chk
 
 
 ORACLE_SAMPLE_TOKENS = 1024
@@ -789,9 +883,11 @@ def main():
                                 device_id=torch.device("cuda", local))
     try:
         res = run_ours(args, world, rank, local)
+        timed = res.pop("_timed_outputs", None)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(args.fwd_only)
-            res["cpu_baseline_all_cores"] = cpu_baseline_all_cores(args.fwd_only)
+            res["cpu_baseline_all_cores"], res["timed_run_check"] = \
+                cpu_baseline_all_cores(args.fwd_only, timed)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

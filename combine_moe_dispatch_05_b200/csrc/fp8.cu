@@ -4,9 +4,13 @@
 // path).  s = amax / 448 in fp32 (1 when the block is all zero), codes =
 // E4M3(x / s) with IEEE fp32 division, round to nearest even, saturating.
 //
-// A half-warp owns one (token, 128-channel) block: 16 lanes x 8 bf16 = one
-// 256-byte row segment read with 16-byte loads, amax reduced by shuffles,
-// 8 codes per lane written as one 8-byte store, one scale per block.
+// A 256-thread CTA owns a token row (grid-stride over tokens): thread i holds
+// 16-byte vectors i, i+256, ... of the bf16 row, four at a time with all four
+// loads issued before any math.  The 16 lanes of a half-warp cover one
+// 128-channel block, reduce its amax with shuffles and convert their 8
+// channels each; pairs of lanes merge their codes into one 16-byte store when
+// q is 16-byte aligned (else each lane stores its 8 codes), and one lane per
+// block writes the scale.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -15,53 +19,65 @@ namespace moe {
 namespace {
 
 constexpr int kQThreads = 256;
+constexpr int kQU = 4;  // columns per thread per batch
 
 __global__ void __launch_bounds__(kQThreads)
 quantize_e4m3_kernel(const uint16_t* __restrict__ x, int64_t T, int H, int64_t stride,
-                     uint8_t* __restrict__ q, float* __restrict__ qs) {
+                     uint8_t* __restrict__ q, float* __restrict__ qs, int vec16) {
   pdl_begin();
-  const int nb = H / 128;
-  const int64_t n_units = T * nb;
-  const int lane = threadIdx.x & 31, sub = lane & 15;
-  const int64_t hw0 = ((int64_t)blockIdx.x * kQThreads + threadIdx.x) >> 4;  // half-warp id
-  const int64_t n_hw = ((int64_t)gridDim.x * kQThreads) >> 4;
-  // both half-warps of a warp run the same number of iterations (shuffles use the full mask)
-  const int64_t hw_even = hw0 & ~(int64_t)1;
-  for (int64_t base = hw_even; base < n_units; base += n_hw) {
-    const int64_t u = base + (hw0 & 1);
-    const bool active = u < n_units;
-    float f[8];
-    float amax = 0.0f;
-    int64_t t = 0, b = 0;
-    if (active) {
-      t = u / nb;
-      b = u - t * nb;
-      const uint4 v = ld_nc_v4(x + t * stride + b * 128 + sub * 8);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const int lane = threadIdx.x & 31;
+  const unsigned half_mask = 0xFFFFu << (lane & 16);
+  const int V = H >> 3;   // 16-byte bf16 vectors per row
+  const int nb = H >> 7;  // 128-channel blocks per row
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    const uint16_t* xr = x + t * stride;
+    uint8_t* qr = q + t * H;
+    for (int vb = threadIdx.x; vb < V; vb += kQThreads * kQU) {  // V % 16 == 0: half-warps stay whole
+      uint4 d[kQU];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        f[2 * i] = bf16_lo(w[i]);
-        f[2 * i + 1] = bf16_hi(w[i]);
+      for (int i = 0; i < kQU; ++i) {
+        const int v = vb + i * kQThreads;
+        d[i] = v < V ? ld_nc_v4(xr + (int64_t)v * 8) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-    }
+      for (int i = 0; i < kQU; ++i) {
+        const int v = vb + i * kQThreads;
+        if (v >= V) break;  // uniform across the half-warp
+        const uint32_t w[4] = {d[i].x, d[i].y, d[i].z, d[i].w};
+        float f[8];
+        float amax = 0.0f;
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o, 16));
-    if (!active) continue;
-    const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-    uint32_t lo = 0, hi = 0;
+        for (int k = 0; k < 4; ++k) {
+          f[2 * k] = bf16_lo(w[k]);
+          f[2 * k + 1] = bf16_hi(w[k]);
+        }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 pr = make_float2(__fdiv_rn(f[2 * i], s), __fdiv_rn(f[2 * i + 1], s));
-      const uint32_t c2 = (uint32_t)__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
-      if (i < 2) lo |= c2 << (16 * i);
-      else hi |= c2 << (16 * (i - 2));
+        for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(f[k]));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)
+          amax = fmaxf(amax, __shfl_xor_sync(half_mask, amax, o, 16));
+        const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        uint32_t c[2] = {0u, 0u};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 pr = make_float2(__fdiv_rn(f[2 * k], s), __fdiv_rn(f[2 * k + 1], s));
+          const uint32_t c2 = (uint32_t)__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
+          c[k >> 1] |= c2 << (16 * (k & 1));
+        }
+        if (vec16) {
+          const uint32_t n0 = __shfl_down_sync(half_mask, c[0], 1, 16);
+          const uint32_t n1 = __shfl_down_sync(half_mask, c[1], 1, 16);
+          if ((lane & 1) == 0) st_v4(qr + (int64_t)v * 8, make_uint4(c[0], c[1], n0, n1));
+        } else {
+          *reinterpret_cast<uint2*>(qr + (int64_t)v * 8) = make_uint2(c[0], c[1]);
+        }
+        if ((lane & 15) == 0) qs[t * nb + (v >> 4)] = s;
+      }
     }
-    *reinterpret_cast<uint2*>(q + t * H + b * 128 + sub * 8) = make_uint2(lo, hi);
-    if (sub == 0) qs[t * nb + b] = s;
   }
 }
+
+std::atomic<int> g_occ_q[moe_host::kMaxCachedDevices];
 
 }  // namespace
 }  // namespace moe
@@ -77,11 +93,12 @@ extern "C" int moe_quantize_e4m3(const void* x, int64_t T, int H, int64_t x_row_
     return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   const int dev = moe_host::current_device();
-  const int64_t units = T * (H / 128);
-  int64_t grid = (units * 16 + moe::kQThreads - 1) / moe::kQThreads;
-  const int64_t cap = (int64_t)moe_host::sm_count(dev) * 8;
-  if (grid > cap) grid = cap;
+  const int bps =
+      moe_host::blocks_per_sm(moe::quantize_e4m3_kernel, moe::kQThreads, 0, dev, moe::g_occ_q);
+  int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
+  if (grid > T) grid = T;
+  const int vec16 = moe_host::aligned16(q) ? 1 : 0;
   return moe_host::launch(moe::quantize_e4m3_kernel, dim3((unsigned)grid), dim3(moe::kQThreads), 0,
                           static_cast<cudaStream_t>(stream), static_cast<const uint16_t*>(x), T, H,
-                          x_row_stride, static_cast<uint8_t*>(q), q_scales);
+                          x_row_stride, static_cast<uint8_t*>(q), q_scales, vec16);
 }

@@ -11,7 +11,7 @@
 // scans, never from the order in which atomics arrive):
 //   1. count:  each 1024-thread block owns a contiguous run of whole tokens
 //      (<= 2048 slots).  Warp w walks its 64-slot segment 32 slots at a time;
-//      __match_any_sync groups the lanes holding the same expert, the
+//      ballots over the id bits group the lanes holding the same expert, the
 //      popcount of the lower lanes is the rank inside the group, and a
 //      per-warp 16-bit shared histogram carries the running count.  A scan
 //      over the 32 warps turns these into each slot's rank inside the block
@@ -36,6 +36,79 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
+}
+
+// Lanes of this warp holding the same valid expert id as this lane (itself
+// included); an invalid lane matches nobody.  One ballot per bit of the id
+// (nbits = bits of E-1, at most 9): two lanes agree on every bit exactly when
+// they hold the same id.
+__device__ __forceinline__ unsigned match_peers(int e, bool valid, int nbits, int lane) {
+  unsigned peers = __ballot_sync(0xffffffffu, valid);
+#pragma unroll
+  for (int b = 0; b < 9; ++b) {
+    if (b < nbits) {
+      const bool bit = (e >> b) & 1;
+      const unsigned m = __ballot_sync(0xffffffffu, bit);
+      peers &= bit ? m : ~m;
+    }
+  }
+  return valid ? peers : (1u << lane);
+}
+
+// One 32-slot step of the count.  rel: the slot's index in the block's run
+// (n_b slots, starting at a token boundary; the warp's steps start at
+// multiples of 32); v: its id.  Validates the id, finds the slot's rank among
+// the earlier slots of the same expert in this warp's segment from the
+// warp's running histogram h, and advances h.  Duplicates inside a token are
+// found from the match when K is a power of two (the token's K slots are one
+// aligned group of K lanes), else by comparing with the token's earlier ids.
+__device__ __forceinline__ void count_step(int rel, int n_b, int v, int K, int E, int nbits,
+                                           const int32_t* s_ids, uint16_t* h, int lane,
+                                           int& err, int& e_out, int& r_out) {
+  const bool k_pow2 = (K & (K - 1)) == 0;
+  int e = -1;
+  if (rel < n_b) {
+    if (v < 0 || v >= E) {
+      if (!err) err = MOE_ERR_EXPERT_RANGE;
+    } else {
+      e = v;
+      if (!k_pow2) {
+        const int k = rel % K;
+        const int base = rel - k;
+        for (int j = 0; j < k; ++j)
+          if (s_ids[base + j] == v && !err) err = MOE_ERR_DUPLICATE_EXPERT;
+      }
+    }
+  }
+  const unsigned peers = match_peers(e, e >= 0, nbits, lane);
+  if (k_pow2 && e >= 0) {
+    const unsigned tok = ((1u << K) - 1u) << (lane & ~(K - 1));  // K <= 16
+    if ((peers & tok & lanemask_lt()) && !err) err = MOE_ERR_DUPLICATE_EXPERT;
+  }
+  int prev = 0;
+  if (e >= 0) prev = h[e];
+  __syncwarp();
+  if (e >= 0 && lane == __ffs(peers) - 1) h[e] = (uint16_t)(prev + __popc(peers));
+  __syncwarp();
+  e_out = e;
+  r_out = e >= 0 ? prev + __popc(peers & lanemask_lt()) : -1;
+}
+
+__device__ __forceinline__ int id_bits(int E) { return E > 1 ? 32 - __clz(E - 1) : 0; }
+
+// dst[0..n) = value, by the threads gt = 0..gs-1: scalar words up to the first
+// 16-byte boundary, 16-byte stores over the body, scalar words after it
+__device__ __forceinline__ void fill_words(uint32_t* dst, int64_t n, uint32_t value, int64_t gt,
+                                           int64_t gs) {
+  int64_t head = (int64_t)((16 - (reinterpret_cast<uintptr_t>(dst) & 15)) & 15) / 4;
+  if (head > n) head = n;
+  if (gt < head) dst[gt] = value;
+  const int64_t nv = (n - head) / 4;
+  uint4* body = reinterpret_cast<uint4*>(dst + head);
+  const uint4 v4 = make_uint4(value, value, value, value);
+  for (int64_t i = gt; i < nv; i += gs) body[i] = v4;
+  const int64_t tail0 = head + nv * 4;
+  if (gt < n - tail0) dst[tail0 + gt] = value;
 }
 
 __global__ void __launch_bounds__(kLayoutThreads)
@@ -67,9 +140,9 @@ layout_count_kernel(const int32_t* __restrict__ ids, int64_t T, int K, int E,
     const int64_t gt = (int64_t)b * kLayoutThreads + tid;
     const int64_t gs = (int64_t)gridDim.x * kLayoutThreads;
     if (row_src)
-      for (int64_t p = gt; p < P_cap; p += gs) row_src[p] = -1;
+      fill_words(reinterpret_cast<uint32_t*>(row_src), P_cap, 0xFFFFFFFFu, gt, gs);
     if (tile_ready)
-      for (int64_t j = gt; j < n_tiles; j += gs) tile_ready[j] = 0u;
+      fill_words(tile_ready, n_tiles, 0u, gt, gs);
   }
   __syncthreads();
 
@@ -77,31 +150,12 @@ layout_count_kernel(const int32_t* __restrict__ ids, int64_t T, int K, int E,
   uint16_t* my_hist = hist + warp * Es;
   int my_e[kItersPerWarp], my_r[kItersPerWarp];
   int err = 0;
+  const int nbits = id_bits(E);
 #pragma unroll
   for (int it = 0; it < kItersPerWarp; ++it) {
     const int rel = warp * (kItersPerWarp * 32) + it * 32 + lane;
-    int e = -1;
-    if (rel < n_b) {
-      const int v = s_ids[rel];
-      if (v < 0 || v >= E) {
-        if (!err) err = MOE_ERR_EXPERT_RANGE;
-      } else {
-        e = v;
-        const int k = rel % K;
-        const int base = rel - k;
-        for (int j = 0; j < k; ++j)
-          if (s_ids[base + j] == v && !err) err = MOE_ERR_DUPLICATE_EXPERT;
-      }
-    }
-    const int key = e >= 0 ? e : -(lane + 1);  // invalid slots match nobody
-    const unsigned grp = __match_any_sync(0xffffffffu, key);
-    int prev = 0;
-    if (e >= 0) prev = my_hist[e];
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(grp) - 1) my_hist[e] = (uint16_t)(prev + __popc(grp));
-    __syncwarp();
-    my_e[it] = e;
-    my_r[it] = e >= 0 ? prev + __popc(grp & lanemask_lt()) : -1;
+    count_step(rel, n_b, rel < n_b ? s_ids[rel] : -1, K, E, nbits, s_ids, my_hist, lane, err,
+               my_e[it], my_r[it]);
   }
   if (err) record_error(status, err);
   __syncthreads();
@@ -276,15 +330,20 @@ extern "C" int moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int K, in
     return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!topk_idx || !dst_row)) return MOE_ERR_INVALID_ARG;
   if (!moe_host::aligned16(workspace)) return MOE_ERR_INVALID_ARG;
+  for (const void* q : {(const void*)topk_idx, (const void*)expert_counts,
+                        (const void*)expert_offsets, (const void*)rank_counts,
+                        (const void*)rank_offsets, (const void*)dst_row, (const void*)row_src,
+                        (const void*)tile_ready})
+    if (!moe_host::aligned4(q)) return MOE_ERR_INVALID_ARG;
   if (workspace_bytes < moe_layout_workspace_bytes(T, K, E)) return MOE_ERR_INVALID_ARG;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t n_tiles = (P_cap + kTile - 1) / kTile;
   const int tpb = tokens_per_block_for(K);
   const int nb = T > 0 ? (int)((T + tpb - 1) / tpb) : 1;
   int32_t* block_counts = static_cast<int32_t*>(workspace);
   int32_t* slot_rank = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
                                                   align256((size_t)nb * E * sizeof(int32_t)));
-  const int64_t n_tiles = (P_cap + kTile - 1) / kTile;
 
   int st = moe_host::launch(layout_count_kernel, dim3(nb), dim3(kLayoutThreads), 0, s, topk_idx, T,
                             K, E, tpb, block_counts, slot_rank, row_src, P_cap, tile_ready,

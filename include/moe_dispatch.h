@@ -121,7 +121,8 @@ MOE_API size_t moe_layout_workspace_bytes(int64_t T, int K, int E);
  *   tile_ready     uint32 [ceil(P_cap/128)] (nullable) chunk-completion
  *                                counters, all set to 0 here
  * Scratch: workspace of workspace_bytes >= moe_layout_workspace_bytes(),
- *   256-byte aligned; its contents need no initialisation.
+ *   256-byte aligned; its contents need no initialisation.  Integer arrays
+ *   must be 4-byte aligned (else MOE_ERR_INVALID_ARG).
  * Data errors: MOE_ERR_EXPERT_RANGE (that slot is not placed),
  *   MOE_ERR_DUPLICATE_EXPERT (both slots are still placed).
  * Results are bit-exact and independent of launch configuration.

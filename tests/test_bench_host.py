@@ -57,3 +57,44 @@ def test_step_bytes_formulas():
 def test_host_cpu_reports_threads_and_model():
     n, model = bench.host_cpu()
     assert n >= 1 and isinstance(model, str) and model
+
+
+def _fake_gpu_outputs(s, res):
+    L = res["layout"]
+    return {"counts": L.counts.copy(), "offsets": L.offsets.copy(),
+            "rank_counts": L.rank_counts.copy(), "rank_offsets": L.rank_offsets.copy(),
+            "dst_row": L.dst_row.copy(), "row_src": L.row_src.copy(),
+            "xp": res["xp"][:L.P].view(np.int16).copy(), "out": res["out"].view(np.int16).copy(),
+            "grad_y": res["grad_y"][:L.P].view(np.int16).copy(),
+            "grad_scales": res["grad_scales"].copy(), "grad_x": res["grad_x"].view(np.int16).copy()}
+
+
+def test_timed_run_check_accepts_identical_and_flags_changes():
+    s = W.config(1)
+    ids, sc = W.topk_ids(s).numpy(), W.topk_scales(s).numpy()
+    x, g = W.as_u16(W.tokens(s)), W.as_u16(W.grad_out(s))
+    _, res = bench.oracle_pass_partitioned(s, ids, sc, x, g, False, 2)
+    ok = bench.check_timed_outputs(s, res, _fake_gpu_outputs(s, res), x, g, False)
+    assert ok["layout_bit_exact"] and ok["permute_bytes_exact"]
+    assert ok["combine_max_ulp"] == 0 and ok["dispatch_bwd_max_ulp"] == 0
+    assert ok["combine_bwd_grad_y_max_ulp"] == 0 and ok["grad_scales_max_err_over_norms"] == 0
+
+    bad = _fake_gpu_outputs(s, res)
+    bad["dst_row"][7] += 1
+    bad["xp"][3, 5] ^= 1
+    bad["out"][2, 9] += 1          # one bf16 ulp (same binade)
+    # three ulps, at an element whose mantissa leaves room inside its binade
+    flat = bad["grad_x"].reshape(-1)
+    i = int(np.flatnonzero((flat.view(np.uint16) & 0x7F) < 0x70)[0])
+    flat[i] += 3
+    chk = bench.check_timed_outputs(s, res, bad, x, g, False)
+    assert not chk["layout_bit_exact"] and not chk["permute_bytes_exact"]
+    assert chk["combine_max_ulp"] == 1 and chk["dispatch_bwd_max_ulp"] == 3
+
+
+def test_bf16_max_ulp_units():
+    one, next_up = np.array([0x3F80], np.uint16), np.array([0x3F81], np.uint16)
+    assert bench.bf16_max_ulp(next_up, one) == 1.0
+    assert bench.bf16_max_ulp(one, one) == 0.0
+    # 2.0 vs 1.0: one unit of 1.0's binade is 2^-7, so the gap is 128 ulps
+    assert bench.bf16_max_ulp(np.array([0x4000], np.uint16), one) == 128.0

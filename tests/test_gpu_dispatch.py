@@ -61,11 +61,35 @@ def test_layout_parity_hot_expert_everywhere():
 
 @pytest.mark.parametrize("T,K,E,R", [
     (1, 1, 1, 1), (0, 4, 8, 2), (1, 16, 16, 4), (63, 3, 5, 5), (65, 8, 512, 8),
-    (1000, 16, 512, 512), (3000, 1, 2, 2), (129, 2, 3, 1), (257, 7, 64, 16), (4097, 6, 64, 16)])
+    (1000, 16, 512, 512), (3000, 1, 2, 2), (129, 2, 3, 1), (257, 7, 64, 16), (4097, 6, 64, 16),
+    # runs of 2048 slots per block: exact multiples and one token past them
+    (4096, 8, 256, 8), (4097, 8, 256, 8), (2048, 16, 512, 8), (2049, 16, 64, 4),
+    (10912, 3, 9, 3), (10913, 3, 9, 3), (700, 5, 40, 8), (3000, 7, 100, 4)])
 def test_layout_parity_edge_shapes(T, K, E, R):
     s = W.Spec("edge", T, 8, E, K, R, "uniform", seed=77 + T + K + E)
     ids = W.topk_ids(s) if T else torch.zeros((0, K), dtype=torch.int32)
     check_layout(ids, E, R)
+
+
+@pytest.mark.parametrize("T,K,E", [(4096, 8, 256), (20000, 8, 256)])
+def test_layout_reuses_buffers_holding_stale_values(T, K, E):
+    """A second call on the same buffers, with garbage left in row_src and
+    tile_ready and different routing, gives exactly the oracle's layout."""
+    s1 = W.Spec("reuse1", T, 8, E, K, 8, "zipf", zipf_s=0.6, seed=901)
+    s2 = W.Spec("reuse2", T, 8, E, K, 8, "zipf", zipf_s=1.2, seed=902)
+    L = ops.moe_dispatch_layout(W.topk_ids(s1).to(DEV), E, 8)
+    L.row_src.fill_(12345)
+    L.tile_ready.fill_(77)
+    L.dst_row.fill_(-9)
+    ids2 = W.topk_ids(s2)
+    st = ops.new_status()
+    ops.moe_dispatch_layout(ids2.to(DEV), E, 8, layout=L, status=st)
+    ref = oracle.layout(ids2.numpy(), E, 8)
+    assert ops.read_status(st) == 0
+    assert np.array_equal(L.expert_offsets.cpu().numpy(), ref.offsets)
+    assert np.array_equal(L.dst_row.cpu().numpy()[:T * K], ref.dst_row)
+    assert np.array_equal(L.row_src.cpu().numpy()[:ref.P_cap], ref.row_src)
+    assert np.all(L.tile_ready.cpu().numpy()[:(ref.P_cap + 127) // 128] == 0)
 
 
 def test_layout_all_tokens_one_expert_multi_tile():
@@ -84,6 +108,23 @@ def test_layout_reports_out_of_range_and_duplicates():
     dup = ids.clone()
     dup[555, 1] = dup[555, 0]
     check_layout(dup, s.E, s.R, expect_status=oracle.ERR_DUPLICATE_EXPERT)
+
+
+@pytest.mark.parametrize("T,K,E", [(300, 8, 64), (9000, 8, 64), (100, 16, 32), (5000, 2, 4),
+                                   (2000, 4, 512), (4096, 8, 256), (700, 5, 40)])
+def test_layout_duplicates_and_range_errors_every_k(T, K, E):
+    """A repeated id inside one token, first at its last slot and then at its
+    second, for K a power of two (found from the lane match) or not (found by
+    comparison), in the first, a middle and the last block."""
+    s = W.Spec("dup", T, 8, E, K, 1, "uniform", seed=5000 + T + K)
+    ids = W.topk_ids(s)
+    for t, j in ((T - 1, K - 1), (T // 2, 1)):
+        dup = ids.clone()
+        dup[t, j] = dup[t, 0]
+        check_layout(dup, E, 1, expect_status=oracle.ERR_DUPLICATE_EXPERT)
+    bad = ids.clone()
+    bad[T // 3, K - 1] = E
+    check_layout(bad, E, 1, expect_status=oracle.ERR_EXPERT_RANGE)
 
 
 # ------------------------------------------------------------ permute ----
@@ -194,7 +235,8 @@ def test_permute_fp8_full_prefill_sampled_rows():
 
 
 # ---------------------------------------------------------- quantiser ----
-@pytest.mark.parametrize("T,H", [(64, 1024), (1000, 7168), (3, 128)])
+@pytest.mark.parametrize("T,H", [(64, 1024), (1000, 7168), (3, 128), (300, 384), (70, 8320),
+                                 (5, 20480)])
 def test_quantize_e4m3_parity(T, H):
     s = W.config(3).with_(T=T, H=H)
     x = W.tokens(s)
@@ -202,6 +244,23 @@ def test_quantize_e4m3_parity(T, H):
     q_ref, s_ref = oracle.quantize_e4m3(W.as_u16(x))
     assert np.array_equal(qs.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def test_quantize_e4m3_strided_rows_and_8_byte_aligned_codes():
+    """x with a row stride wider than H, and a code buffer that is only
+    8-byte aligned (each lane stores its own 8 codes)."""
+    s = W.config(3).with_(T=257, H=640)
+    x = W.tokens(s)
+    wide = torch.zeros((s.T, s.H + 24), dtype=torch.bfloat16)
+    wide[:, 16:16 + s.H] = x
+    xd = wide.to(DEV)[:, 16:16 + s.H]
+    flat = torch.full((s.T * s.H + 8,), 0xA5, dtype=torch.uint8, device=DEV)
+    q = flat[8:].view(s.T, s.H)
+    q, qs = ops.moe_quantize_e4m3(xd, q=q)
+    q_ref, s_ref = oracle.quantize_e4m3(W.as_u16(x))
+    assert np.array_equal(qs.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert int(flat[:8].to(torch.int32).sum()) == 8 * 0xA5
 
 
 def test_quantize_then_dispatch_fp8_pipeline():
