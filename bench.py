@@ -498,11 +498,44 @@ def e2e(args, ops, torch, dev, stream, L, host_in, dev_in, bufs, flush, T, K, E,
     end.synchronize()
     tot = max_over_ranks(start.elapsed_time(end), world)
     ms = tot / args.steps
-    return {"value": round(bytes_step * world / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
-            "ms_per_step": round(ms, 4), "tokens_per_s": round(T * world / (ms * 1e-3), 1),
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "overlap": "copies on separate streams, two alternating buffer sets",
-            "l2": "not flushed: each step moves ~3.2 GB through HBM, far beyond L2"}
+    res = {"value": round(bytes_step * world / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+           "ms_per_step": round(ms, 4), "tokens_per_s": round(T * world / (ms * 1e-3), 1),
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "overlap": "copies on separate streams, two alternating buffer sets",
+           "l2": "not flushed: each step moves ~3.2 GB through HBM, far beyond L2"}
+    if world == 1:
+        # the copies alone, both directions at once on the same streams: the
+        # PCIe bound of this end-to-end step (no kernels)
+        b = sets[0]
+        pairs_in = [(b["ids"], ids_h), (b["sc"], sc_h), (b["x"], x_h)] + \
+            ([] if args.fwd_only else [(b["g"], g_h)])
+        pairs_out = [(b["out_h"], b["out"])] + \
+            ([] if args.fwd_only else [(b["gx_h"], b["gx"]), (b["gs_h"], b["gs"])])
+
+        def copies():
+            with torch.cuda.stream(h2d_s):
+                for d, h in pairs_in:
+                    d.copy_(h, non_blocking=True)
+            with torch.cuda.stream(d2h_s):
+                for h, d in pairs_out:
+                    h.copy_(d, non_blocking=True)
+        copies()
+        torch.cuda.synchronize()
+        n = min(args.steps, 20)
+        start.record(comp)
+        h2d_s.wait_stream(comp)
+        d2h_s.wait_stream(comp)
+        for _ in range(n):
+            copies()
+        comp.wait_stream(h2d_s)
+        comp.wait_stream(d2h_s)
+        end.record(comp)
+        end.synchronize()
+        copy_ms = start.elapsed_time(end) / n
+        res["copies_only_ms_per_step"] = round(copy_ms, 4)
+        res["pcie_gbps_per_direction"] = round(max(h2d, d2h) / (copy_ms * 1e-3) / 1e9, 1)
+        res["frac_of_copy_bound"] = round(copy_ms / ms, 4)
+    return res
 
 
 # ------------------------------------------------------ other workloads --
