@@ -413,7 +413,8 @@ extern "C" int moe_combine_bwd(const void* grad_out, const void* y, const float*
   using namespace moe;
   int st = check_rows_args(y, dst_row, T, K, H, P_cap, grad_y);
   if (st != MOE_OK) return st;
-  if (E < 1 || E > MOE_MAX_EXPERTS || !expert_counts || !expert_offsets || !grad_y)
+  if (E < 1 || E > MOE_MAX_EXPERTS || !expert_counts || !expert_offsets ||
+      (P_cap > 0 && !grad_y))
     return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!grad_out || !scales || !grad_scales)) return MOE_ERR_INVALID_ARG;
   if (grad_out && !moe_host::aligned16(grad_out)) return MOE_ERR_INVALID_ARG;

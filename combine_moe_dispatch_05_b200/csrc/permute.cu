@@ -698,12 +698,14 @@ int make_perm_args(const void* x, int dtype, int64_t T, int H, int64_t x_row_str
   const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 1;
   const int64_t row_bytes = (int64_t)H * elem;
   if (row_bytes % 16 != 0 || (x_row_stride * elem) % 16 != 0) return MOE_ERR_INVALID_ARG;
-  if (!xp || !expert_counts || !expert_offsets || (T > 0 && (!x || !dst_row)))
+  // an empty batch (P_cap = 0) may pass null row buffers
+  if ((P_cap > 0 && !xp) || !expert_counts || !expert_offsets || (T > 0 && (!x || !dst_row)))
     return MOE_ERR_INVALID_ARG;
   if (!moe_host::aligned16(xp) || (x && !moe_host::aligned16(x))) return MOE_ERR_INVALID_ARG;
   int scale_cols = 0;
   if (dtype == MOE_DTYPE_E4M3) {
-    if (H % 128 != 0 || !xp_scales || (T > 0 && !x_scales)) return MOE_ERR_INVALID_ARG;
+    if (H % 128 != 0 || (P_cap > 0 && !xp_scales) || (T > 0 && !x_scales))
+      return MOE_ERR_INVALID_ARG;
     scale_cols = H / 128;
     if (x_scales_row_stride < scale_cols) return MOE_ERR_INVALID_ARG;
   } else if (x_scales || xp_scales) {

@@ -242,7 +242,9 @@ extern "C" int moe_dispatch_permute_quant(const void* x, int64_t T, int H, int64
     return MOE_ERR_INVALID_ARG;
   if (T * (int64_t)K > (int64_t)INT32_MAX || P_cap > (int64_t)INT32_MAX) return MOE_ERR_INVALID_ARG;
   if (P_cap < moe_padded_capacity(T, K, E)) return MOE_ERR_CAPACITY;
-  if (!xp || !xp_scales || !expert_counts || !expert_offsets || (T > 0 && (!x || !dst_row)))
+  // an empty batch (P_cap = 0) may pass null row buffers
+  if ((P_cap > 0 && (!xp || !xp_scales)) || !expert_counts || !expert_offsets ||
+      (T > 0 && (!x || !dst_row)))
     return MOE_ERR_INVALID_ARG;
   if (!moe_host::aligned16(xp) || (x && !moe_host::aligned16(x)) || !moe_host::aligned4(xp_scales))
     return MOE_ERR_INVALID_ARG;

@@ -32,6 +32,9 @@
  *     enqueued on it; no call synchronises the host.
  *   - bf16 = IEEE bfloat16 (2 bytes), E4M3 = OCP 8-bit float E4M3 (1 byte).
  *   - Row-major layouts; "[A, B]" = A rows of B elements.
+ *   - Empty batch (T = 0): the layout writes zero counts and offsets; every
+ *     other call returns MOE_OK without a launch.  Buffers that have no rows
+ *     in that case (x, xp, xp_scales, grad_y, out, ...) may be NULL.
  *   - Return value: MOE_OK if the work was enqueued.  Argument errors that
  *     the host can see (NULL where not allowed, sizes out of range, bad
  *     alignment, E % R != 0, capacity too small) return at once and launch

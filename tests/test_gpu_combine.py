@@ -196,3 +196,43 @@ def test_combine_strict_one_ulp_on_workloads(cfg, shared):
     err = np.abs(f64(dev_u16(out)) - exact)
     over = err > 2.0 ** -7 * np.abs(exact)
     assert over.mean() < 1e-5, (int(over.sum()), over.size)
+
+
+def test_combine_and_backward_full_prefill_sampled_tokens():
+    """Full prefill size (T=32768, H=7168, K=8: 2.2 M rows of bf16 expert
+    outputs) in the launch configuration the benchmark uses; 256 sampled
+    tokens are checked against the oracle, which sees only their rows."""
+    s = W.config(3)
+    ids = W.topk_ids(s).to(DEV)
+    st = ops.new_status()
+    L = ops.moe_dispatch_layout(ids, s.E, s.R, status=st)
+    y = W.expert_out(s, L.P_cap, device=DEV)
+    g = W.grad_out(s, device=DEV)
+    sc = W.topk_scales(s).to(DEV)
+    out = ops.moe_combine(y, L.dst_row, sc, status=st)
+    gy, gs = ops.moe_combine_bwd(g, y, sc, L, status=st)
+    gx = ops.moe_dispatch_bwd(gy, L.dst_row, s.T, s.K, status=st)
+    assert ops.read_status(st) == 0
+    tok = torch.randperm(s.T, generator=torch.Generator().manual_seed(3))[:256].to(DEV)
+    rows = L.dst_row.view(s.T, s.K)[tok].long()                   # [n, K]
+    n = tok.numel()
+    y_s = W.as_u16(y[rows.reshape(-1)].cpu())                      # the sampled rows only
+    g_s = W.as_u16(g[tok].cpu())
+    local = np.arange(n * s.K, dtype=np.int32)                     # row i of y_s
+    sc_s = sc[tok].cpu().numpy()
+    ref = oracle.combine(y_s, local, sc_s, None)
+    assert_bf16_close(dev_u16(out[tok]), ref, combine_mag(y_s, local, sc_s), s.K, "combine")
+    counts = np.zeros(1, np.int32)
+    offs = np.zeros(2, np.int32)                                   # no padding rows here
+    gy_ref = np.zeros((n * s.K, s.H), np.uint16)
+    gs_ref = oracle.combine_bwd(g_s, y_s, sc_s, local, counts, offs, gy_ref)
+    got_gy = dev_u16(gy[rows.reshape(-1)])
+    assert_bf16_close(got_gy, gy_ref, np.abs(f64(gy_ref)), 1, "grad_y")
+    dmag = np.einsum("th,tkh->tk", np.abs(f64(g_s)), np.abs(f64(y_s)).reshape(n, s.K, s.H))
+    err = np.abs(gs[tok].cpu().numpy().astype(np.float64) - gs_ref.astype(np.float64))
+    assert np.all(err <= gamma(s.H) * dmag + 2.0 ** -24 * np.abs(gs_ref) + 1e-30)
+    # dispatch_bwd read the GPU's grad_y: the oracle sums those same rows
+    gx_ref = oracle.dispatch_bwd(got_gy, local, n, s.K)
+    ones = np.ones((n, s.K), np.float32)
+    assert_bf16_close(dev_u16(gx[tok]), gx_ref, combine_mag(got_gy, local, ones), s.K,
+                      "dispatch_bwd")
