@@ -755,6 +755,28 @@ int optin_smem(int dev) {
   return optin;
 }
 
+// Lets `kernel` request up to all the dynamic shared memory the device
+// allows, once per device.  (Setting the exact size of each call instead
+// would race between host threads launching different row sizes.)  The
+// occupancy still follows the size each launch asks for.
+template <typename F>
+bool allow_max_dyn_smem(F kernel, int dev, int optin, std::atomic<int>* done) {
+  const bool cached = dev >= 0 && dev < moe_host::kMaxCachedDevices;
+  if (cached && done[dev].load(std::memory_order_acquire)) return true;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess ||
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin - (int)fa.sharedSizeBytes) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (cached) done[dev].store(1, std::memory_order_release);
+  return true;
+}
+
+std::atomic<int> g_dyn_perm[moe_host::kMaxCachedDevices];
+std::atomic<int> g_dyn_consume[moe_host::kMaxCachedDevices];
+
 }  // namespace
 }  // namespace moe
 
@@ -778,9 +800,7 @@ extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
   const int ctas_per_sm = perm_ctas_per_sm(a.row_bytes);
   const size_t dyn = size_ring(a, ctas_per_sm, sizeof(PermShared), optin);
   if (dyn == 0) return MOE_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)dyn) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (!allow_max_dyn_smem(permute_kernel, dev, optin, g_dyn_perm)) return MOE_ERR_CUDA;
 
   const int64_t v_bound = T * K + (int64_t)(kTile - 1) * E;
   int64_t grid = (int64_t)moe_host::sm_count(dev) * ctas_per_sm;
@@ -814,9 +834,7 @@ extern "C" int moe_dispatch_permute_consume(
   const size_t static_smem = sizeof(TileShared) + 64;
   const size_t dyn = size_ring(a, kFusedCtasPerSm, static_smem, optin);
   if (dyn == 0) return MOE_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(permute_consume_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)dyn) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (!allow_max_dyn_smem(permute_consume_kernel, dev, optin, g_dyn_consume)) return MOE_ERR_CUDA;
   // every CTA must be resident at once (consumers wait on other CTAs' rows):
   // a cooperative launch no larger than the device can hold
   int per_sm = 0;
