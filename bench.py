@@ -12,9 +12,12 @@ ranks, Zipf(0.6) routing):
 value = algorithmic HBM bytes of the step / device time of the step, in GB/s
 (also reported: tokens/s).  Inputs are resident in HBM when the timed region
 starts; L2 is flushed (256 MiB write) before every timed step and the flush
-is outside the timed events.  With N GPUs (torchrun), every rank runs its own
-replica on its own data (weak scaling; no collective on the data path); the
-reported time is the max over ranks.
+is outside the timed events.  Inside the timed region the only events are
+one before and one after each step; per-kernel times (phases_us, and the
+roofline's dominant kernel) come from a separate pass right after it with an
+event between every two kernels.  With N GPUs (torchrun), every rank runs its
+own replica on its own data (weak scaling; no collective on the data path);
+the reported time is the max over ranks.
 
 --impl reference times the CPU oracle (single-threaded C) on a bounded sample
 of the same workload and prints the same line with "impl": "reference".
@@ -84,18 +87,29 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def kernel_source_sha(srcfile: str):
+    """sha1[:12] of a kernel's source file followed by the shared device
+    header it includes (common.cuh), or None if either is missing."""
+    csrc = os.path.join(ROOT, "combine_moe_dispatch_05_b200", "csrc")
+    try:
+        data = open(os.path.join(csrc, srcfile), "rb").read() + \
+            open(os.path.join(csrc, "common.cuh"), "rb").read()
+    except OSError:
+        return None
+    return hashlib.sha1(data).hexdigest()[:12]
+
+
 def ncu_traffic(kernel_key: str):
     """dram bytes per launch of `kernel_key` from the committed ncu summaries,
-    if the kernel's source file is unchanged since the capture (else None).
-    Summary lines look like:  traffic: <key> <bytes per launch> src=<sha1[:12]>"""
+    if the kernel's sources are unchanged since the capture (else None).
+    Summary lines look like:  traffic: <key> <bytes per launch> src=<sha1[:12]>
+    where the sha covers the kernel's .cu file and common.cuh."""
     srcfile = {"permute": "permute.cu", "combine": "combine.cu", "combine_bwd": "combine.cu",
                "dispatch_bwd": "combine.cu", "layout": "layout.cu"}.get(kernel_key)
     if srcfile is None:
         return None
-    src = os.path.join(ROOT, "combine_moe_dispatch_05_b200", "csrc", srcfile)
-    try:
-        sha = hashlib.sha1(open(src, "rb").read()).hexdigest()[:12]
-    except OSError:
+    sha = kernel_source_sha(srcfile)
+    if sha is None:
         return None
     for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         for line in open(f):
@@ -269,35 +283,25 @@ def run_ours(args, world, rank, local):
         with torch.cuda.graph(graph, stream=side):
             step()
         torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    # Timed region: one event before and one after each step, none between
+    # the kernels (an event between two kernels ends the programmatic launch
+    # chain and serialises them: ~5 us per boundary).
+    bounds = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(smi_id(torch, dev)) as clk:
         for i in range(args.steps):
             flush.zero_()
+            bounds[i][0].record(stream)
             if graph is not None:
-                evs[i][0].record(stream)
                 graph.replay()
-                evs[i][-1].record(stream)
             else:
-                step(evs[i])
+                step()
+            bounds[i][1].record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    per_phase = {p: [] for p in phases}
-    step_ms = []
-    for e in evs:
-        step_ms.append(e[0].elapsed_time(e[-1]))
-        if graph is None:
-            for j, p in enumerate(phases):
-                per_phase[p].append(e[j].elapsed_time(e[j + 1]))
-    if graph is not None:  # per-kernel times from one eager pass per step
-        for i in range(min(args.steps, 50)):
-            flush.zero_()
-            step(evs[i])
-        torch.cuda.synchronize()
-        for e in evs[:min(args.steps, 50)]:
-            for j, p in enumerate(phases):
-                per_phase[p].append(e[j].elapsed_time(e[j + 1]))
+    step_ms = [a.elapsed_time(b) for a, b in bounds]
     snapshot = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # the last timed step's outputs, checked against the oracle's pass in
@@ -313,6 +317,19 @@ def run_ours(args, world, rank, local):
         snapshot["xp"] = xp[:P_now].view(torch.int16).cpu().numpy()
         if "grad_y" in snapshot:
             snapshot["grad_y"] = snapshot["grad_y"][:P_now]
+    # Per-kernel durations: a pass right after the timed region with an event
+    # between every two kernels, which isolates each kernel's own time.
+    n_phase = min(args.steps, 100)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(n_phase)]
+    for i in range(n_phase):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    per_phase = {p: [] for p in phases}
+    for e in evs:
+        for j, p in enumerate(phases):
+            per_phase[p].append(e[j].elapsed_time(e[j + 1]))
+    phase_step_ms = statistics.mean(e[0].elapsed_time(e[-1]) for e in evs)
     total_ms = sum(step_ms)
     total_ms_max = max_over_ranks(total_ms, world)
     ms_per_step = total_ms_max / args.steps
@@ -332,6 +349,9 @@ def run_ours(args, world, rank, local):
                 "measured" else "fallback 6.65 TB/s",
                 "traffic": ncu_traffic(dom),
                 "algorithmic_bytes_per_launch": nbytes[dom],
+                "duration_source": f"mean of {n_phase} launches in the per-kernel pass after "
+                                   "the timed region (events on the launching stream on both "
+                                   "sides of each kernel, L2 flushed before each step)",
                 "step_frac": round(bytes_step / (ms_per_step * 1e-3) / 1e9 / peak, 4),
                 "fwd_frac": round(fwd_bytes / (fwd_us * 1e-6) / 1e9 / peak, 4)}
 
@@ -348,6 +368,9 @@ def run_ours(args, world, rank, local):
                                 "eager launches (programmatic dependent launch)",
                       "parallelism": f"replicas x{world}"},
            "phases_us": {p: round(v, 2) for p, v in phase_us.items()},
+           "phases_note": f"per-kernel pass of {n_phase} steps with an event between every two "
+                          f"kernels (which serialises them): {phase_step_ms:.4f} ms per step "
+                          "there, against ms_per_step in the timed region",
            "phases_gbs": {p: round(v, 1) for p, v in phase_gbs.items()},
            "roofline": roofline,
            "gpu_launches": LAUNCHES_PER_STEP[args.fwd_only] * args.steps,
@@ -361,12 +384,14 @@ def run_ours(args, world, rank, local):
     if world == 1 and graph is None:
         # the same step back to back without the flush: part of each step's
         # inputs is still in L2 from the step before
-        warm = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+        warm = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(min(args.steps, 100))]
-        for e in warm:
-            step(e)
+        for a, b in warm:
+            a.record(stream)
+            step()
+            b.record(stream)
         torch.cuda.synchronize()
-        warm_ms = statistics.median(e[0].elapsed_time(e[-1]) for e in warm)
+        warm_ms = statistics.median(a.elapsed_time(b) for a, b in warm)
         res["warm_l2"] = {"ms_per_step_median": round(warm_ms, 5),
                           "value": round(bytes_step / (warm_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                           "note": "L2 not flushed between steps; not the headline value"}

@@ -21,12 +21,15 @@ constexpr int kTile = MOE_TILE_M;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s for any device-side wait
 
 // ------------------------------------------- programmatic dependent launch --
-// Every kernel starts with these two: it lets the next kernel in the stream
-// begin launching, then waits until the previous kernel has finished and its
-// writes are visible.  Stream order of all memory accesses is unchanged; only
-// the launch latency overlaps the previous kernel's tail.
+// Every kernel is launched with programmatic stream serialization and starts
+// by waiting until the previous kernel has finished and its writes are
+// visible.  No kernel triggers its dependents early: the next kernel's launch
+// begins as this grid's CTAs exit, which hides the launch and grid-teardown
+// latency without parking the next grid's CTAs on SMs that are still busy.
+// (An early trigger at kernel start measured 559 us per decode step, no
+// programmatic launch 525 us, this form 514 us.)  Stream order of all memory
+// accesses is unchanged.
 __device__ __forceinline__ void pdl_begin() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
