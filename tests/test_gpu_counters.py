@@ -114,6 +114,19 @@ def test_bounds_guard_skips_rows_outside_the_buffer():
                         status=st)
     assert ops.read_status(st) == ops.ERR_BOUNDS
     assert bool((guard[L.P_cap:].view(torch.int16) == 0x1234).all())
+    # E4M3 rows: the byte permute and the fused quantise-dispatch
+    gq = torch.full((L.P_cap + 64, s.H), 0x77, dtype=torch.uint8, device=DEV)
+    gqs = torch.full((L.P_cap + 64, s.H // 128), -5.0, dtype=torch.float32, device=DEV)
+    st = ops.new_status()
+    ops.moe_dispatch_permute(W.e4m3_codes(s).to(DEV), L, xp=gq[:L.P_cap],
+                             x_scales=W.block_scales(s).to(DEV), xp_scales=gqs[:L.P_cap],
+                             status=st)
+    assert ops.read_status(st) == ops.ERR_BOUNDS
+    st = ops.new_status()
+    ops.moe_dispatch_permute_quant(W.tokens(s).to(DEV), L, xp=gq[:L.P_cap],
+                                   xp_scales=gqs[:L.P_cap], status=st)
+    assert ops.read_status(st) == ops.ERR_BOUNDS
+    assert bool((gq[L.P_cap:] == 0x77).all()) and bool((gqs[L.P_cap:] == -5.0).all())
 
 
 def test_out_of_range_ids_are_skipped_downstream():
