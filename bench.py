@@ -420,6 +420,8 @@ def run_ours(args, world, rank, local):
                           "us": {k: round(v, 1) for k, v in t.items()},
                           "gain": round(1 - t["layout_permute_with_concurrent_consumer"] /
                                         t["layout_permute_then_consumer"], 3)}
+        res["shared_expert_overlap"] = shared_expert_overlap(ops, torch, dev, flush, stream, ids,
+                                                             sc, x, L, xp, E, R)
         res["other_workloads"] = extra_workloads(args, dev, flush, stream)
         res["planner"] = plan_on(L, E, R, ops)
 
@@ -582,6 +584,63 @@ def time_calls(torch, calls, flush, steps, stream):
             ts.append(a.elapsed_time(b) * 1e3)
         out[name] = statistics.median(ts)
     return out
+
+
+def shared_expert_overlap(ops, torch, dev, flush, stream, ids, sc, x, L, xp, E, R):
+    """Shared-expert work on a second stream while the dispatch runs.
+
+    Stand-in for the shared expert: a dense MLP on every token,
+    shared_x = silu(x @ W1) @ W2 with DeepSeek-V3's shared-expert width
+    (2048), done by torch matmuls (cuBLAS); it is not part of this library.
+    Sequential: layout, permute, shared MLP, combine(+shared_x) on one stream.
+    Overlapped: the shared MLP runs on a second stream from the start of the
+    step; combine waits for both.  Medians of 20 runs, L2 flushed before
+    each; the two combine outputs must be identical."""
+    T, H = x.shape
+    g = torch.Generator(device=dev).manual_seed(20260100)
+    w1 = (torch.randn((H, 2048), generator=g, device=dev) * H ** -0.5).to(torch.bfloat16)
+    w2 = (torch.randn((2048, H), generator=g, device=dev) * 2048 ** -0.5).to(torch.bfloat16)
+    sh = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    hid = torch.empty((T, 2048), dtype=torch.bfloat16, device=dev)
+    outs = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    st = ops.new_status(dev)
+    side = torch.cuda.Stream(device=dev)
+
+    def mlp():
+        torch.matmul(x, w1, out=hid)
+        torch.nn.functional.silu(hid, inplace=True)
+        torch.matmul(hid, w2, out=sh)
+
+    def sequential():
+        ops.moe_dispatch_layout(ids, E, R, layout=L, status=st)
+        ops.moe_dispatch_permute(x, L, xp=xp, status=st)
+        mlp()
+        ops.moe_combine(xp, L.dst_row, sc, shared_x=sh, out=outs[0], status=st)
+
+    def overlapped():
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            mlp()
+        ops.moe_dispatch_layout(ids, E, R, layout=L, status=st)
+        ops.moe_dispatch_permute(x, L, xp=xp, status=st)
+        stream.wait_stream(side)
+        ops.moe_combine(xp, L.dst_row, sc, shared_x=sh, out=outs[1], status=st)
+
+    t = time_calls(torch, [("mlp_alone", mlp), ("layout_permute", lambda: (
+        ops.moe_dispatch_layout(ids, E, R, layout=L, status=st),
+        ops.moe_dispatch_permute(x, L, xp=xp, status=st))),
+        ("sequential", sequential), ("overlapped", overlapped)], flush, 20, stream)
+    torch.cuda.synchronize()
+    if ops.read_status(st) != 0:
+        raise RuntimeError(f"device status {ops.read_status(st)} in the shared-expert runs")
+    flops = 2 * 2 * T * H * 2048
+    return {"what": "layout + permute with a shared-expert MLP stand-in (x @ W1 -> silu -> @ W2, "
+                    "width 2048, torch/cuBLAS bf16) on a second stream, then combine with "
+                    "shared_x",
+            "us": {k: round(v, 1) for k, v in t.items()},
+            "mlp_tflops": round(flops / (t["mlp_alone"] * 1e-6) / 1e12, 1),
+            "gain": round(1 - t["overlapped"] / t["sequential"], 3),
+            "outputs_identical": bool(torch.equal(outs[0], outs[1]))}
 
 
 def extra_workloads(args, dev, flush, stream):
