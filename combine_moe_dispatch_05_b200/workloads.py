@@ -27,7 +27,6 @@ chosen experts.
 from __future__ import annotations
 
 import dataclasses
-from typing import Optional
 
 import numpy as np
 import torch

@@ -4,7 +4,6 @@ seeded inputs, and the tolerances the comparisons use."""
 import numpy as np
 import torch
 
-import oracle
 from combine_moe_dispatch_05_b200 import build as B
 from combine_moe_dispatch_05_b200 import ops
 from combine_moe_dispatch_05_b200 import workloads as W

@@ -5,7 +5,6 @@ import glob
 import os
 import re
 
-import pytest
 
 from combine_moe_dispatch_05_b200 import build as B
 from combine_moe_dispatch_05_b200 import ops

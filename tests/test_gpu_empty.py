@@ -1,7 +1,6 @@
 """An empty batch (T = 0) through every call: the layout reports zero
 counts and offsets, every other call succeeds without writing anything, and
 buffers without rows may be empty tensors (NULL pointers at the C ABI)."""
-import numpy as np
 import pytest
 import torch
 

@@ -2,7 +2,6 @@
 launched with programmatic stream serialization, which graphs keep; replays
 on new inputs (copied into the captured buffers) must give exactly what eager
 calls give."""
-import numpy as np
 import pytest
 import torch
 

@@ -14,8 +14,6 @@ import shutil
 import subprocess
 import sys
 
-import pytest
-
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
 PINS = ["tests/test_oracle_dispatch.py", "tests/test_oracle_combine.py",

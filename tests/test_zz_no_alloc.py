@@ -14,7 +14,6 @@ already run every other test.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
