@@ -56,7 +56,8 @@ def run(s, strided=False, scales_offset=0):
                                        (50, 128, 3, 2, 1), (1, 128, 1, 1, 1),
                                        (700, 1152, 512, 16, 8), (129, 896, 7, 7, 7),
                                        (90, 20480, 16, 4, 4), (61, 8704, 9, 3, 3),
-                                       (75, 8320, 6, 5, 2), (5000, 1024, 4, 2, 2)])
+                                       (75, 8320, 6, 5, 2), (5000, 1024, 4, 2, 2),
+                                       (8192, 7168, 256, 8, 8)])
 def test_fused_quant_dispatch_matches_oracle(T, H, E, K, R):
     run(W.config(3).with_(T=T, H=H, E=E, K=K, R=R))
 
