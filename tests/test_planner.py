@@ -62,6 +62,47 @@ def test_golden_affinity_prefers_expert_already_on_dst():
     assert after < before
 
 
+def test_golden_tile_term_and_rounded_up_tiles():
+    # t = max(b2*(tiles - G), 0.1*N).  rank0 = {e1: 200}: tiles 2, G 1 -> 100;
+    # rank1 = {e3: 128, e4: 256, e5: 512}: tiles 1+2+4 = 7, G 3 -> 400.
+    # Water-filling takes e5 (largest, none on dst): 4 and 3 chunks leave dst
+    # dearer than src; 2 chunks give 200 | 200 (tiles 2+2 on rank0, 1+2+2 on
+    # rank1).  Then both ranks cost 200 and the planner stops.
+    cost = OP.Cost(a=0, b=0, b2=100.0, c=0, beta=0.1, mig=0)
+    moves, before, after, _ = OP.plan([0, 200, 0, 128, 256, 512], 2, cost)
+    assert (moves, before, after) == ([(5, 1, 0, 256)], 400.0, 200.0)
+
+
+def test_golden_affinity_decides_the_second_move():
+    # t = max(40*(tiles - G), N).  Start 1600 | 640.  Move 1: e1 (700, first
+    # of the tied largest) gives 3 chunks: 1216 | 1024.  Move 2: e1 is now on
+    # rank 1, so it is tried before the larger e2; one chunk of it (no larger
+    # split keeps dst <= src) gives 1088 | 1152, below 1216, and is kept.
+    # Moving e2 instead would also have passed the guard; affinity picks e1.
+    # Nothing after that lowers 1152.
+    cost = OP.Cost(a=0, b=0, b2=40.0, c=0, beta=1.0, mig=0)
+    moves, before, after, _ = OP.plan([200, 700, 700, 512, 0, 128], 2, cost)
+    assert (moves, before, after) == ([(1, 0, 1, 384), (1, 0, 1, 128)], 1600.0, 1152.0)
+
+
+def test_golden_single_chunk_when_no_split_fits():
+    # t = max(500*G, N).  1000 | 1536.  From rank 1 (e3: 1024, e2: 512) no
+    # number of e3's chunks leaves rank 0 (which gains a third replica: 1500)
+    # no dearer than rank 1, so one chunk is tried: 1500 | 1408 -> kept.
+    # Every later single-chunk move leaves some rank at 1500 or more.
+    cost = OP.Cost(a=0, b=500.0, b2=0, c=0, beta=1.0, mig=0)
+    moves, before, after, _ = OP.plan([384, 512, 512, 1024], 2, cost)
+    assert (moves, before, after) == ([(3, 1, 0, 128)], 1536.0, 1500.0)
+
+
+def test_fine_chunk_is_one_tile_or_the_remainder():
+    cost = OP.Cost()
+    loads = [{0: 300}, {}]
+    assert OP._chunk_for(loads, [0, 0], cost, 0, 1, 0, True) == 128
+    loads = [{0: 77}, {}]
+    assert OP._chunk_for(loads, [0, 0], cost, 0, 1, 0, True) == 77
+
+
 @pytest.mark.parametrize("seed", range(25))
 def test_oracle_invariants_and_independent_cost(seed):
     rng = np.random.default_rng(seed)
@@ -147,6 +188,19 @@ def test_library_planner_matches_oracle(_lib, seed):
                                       cost.mig, min_gain=min_gain, max_moves=64)
     assert lm == moves
     assert lb == before and la == after       # bit-identical doubles
+
+
+@pytest.mark.parametrize("counts,R,cost,expect", [
+    ([0, 200, 0, 128, 256, 512], 2, dict(b=0.0, b2=100.0, beta=0.1),
+     ([(5, 1, 0, 256)], 400.0, 200.0)),
+    ([200, 700, 700, 512, 0, 128], 2, dict(b=0.0, b2=40.0, beta=1.0),
+     ([(1, 0, 1, 384), (1, 0, 1, 128)], 1600.0, 1152.0)),
+    ([384, 512, 512, 1024], 2, dict(b=500.0, b2=0.0, beta=1.0), ([(3, 1, 0, 128)], 1536.0, 1500.0)),
+    ([1024, 0, 0, 0], 2, dict(b=0.0, b2=0.0, beta=1.0), ([(0, 0, 1, 512)], 1024.0, 512.0))])
+def test_library_planner_hand_worked_plans(_lib, counts, R, cost, expect):
+    """The hand-worked plans of the oracle pins above, from the C++ planner."""
+    lm, lb, la = ops.moe_plan_balance(counts, R, a=0.0, c=0.0, mig=0.0, **cost)
+    assert (lm, lb, la) == expect
 
 
 def test_library_planner_on_decode_workload(_lib):
