@@ -220,6 +220,8 @@ def moe_dispatch_permute(x: torch.Tensor, L: Layout, xp: Optional[torch.Tensor] 
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be 2-D with unit column stride")
     T, H = x.shape
+    if T != L.T:
+        raise ValueError(f"x has {T} rows but the layout was built for {L.T} tokens")
     if x.dtype == torch.bfloat16:
         dt, el = DTYPE_BF16, torch.bfloat16
     elif x.dtype in (torch.uint8, torch.float8_e4m3fn):
@@ -257,6 +259,8 @@ def moe_dispatch_permute_consume(x: torch.Tensor, L: Layout, xp: Optional[torch.
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be 2-D with unit column stride")
     T, H = x.shape
+    if T != L.T:
+        raise ValueError(f"x has {T} rows but the layout was built for {L.T} tokens")
     if x.dtype == torch.bfloat16:
         dt = DTYPE_BF16
     elif x.dtype in (torch.uint8, torch.float8_e4m3fn):
@@ -296,6 +300,8 @@ def moe_dispatch_permute_quant(x: torch.Tensor, L: Layout, xp: Optional[torch.Te
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be 2-D with unit column stride")
     T, H = x.shape
+    if T != L.T:
+        raise ValueError(f"x has {T} rows but the layout was built for {L.T} tokens")
     if xp is None:
         xp = torch.empty((L.P_cap, H), dtype=torch.uint8, device=x.device)
     if xp_scales is None:
@@ -320,8 +326,12 @@ def moe_combine(y: torch.Tensor, dst_row: torch.Tensor, scales: torch.Tensor,
     _cuda(scales, "scales", torch.float32)
     T, K = scales.shape
     H = y.shape[1]
+    if dst_row.numel() < T * K:
+        raise ValueError(f"dst_row has {dst_row.numel()} entries, needs T*K = {T * K}")
+    if P_cap is not None and P_cap > y.shape[0]:
+        raise ValueError(f"P_cap={P_cap} exceeds the {y.shape[0]} rows of y")
     if shared_x is not None:
-        _cuda(shared_x, "shared_x", torch.bfloat16)
+        _shape(_cuda(shared_x, "shared_x", torch.bfloat16), "shared_x", (T, H))
     if out is None:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
     _shape(_cuda(out, "out", torch.bfloat16), "out", (T, H))
@@ -341,6 +351,12 @@ def moe_combine_bwd(grad_out: torch.Tensor, y: torch.Tensor, scales: torch.Tenso
     _cuda(scales, "scales", torch.float32)
     T, K = scales.shape
     H = grad_out.shape[1]
+    _shape(grad_out, "grad_out", (T, H))
+    if (T, K) != (L.T, L.K):
+        raise ValueError(f"scales is {T}x{K} but the layout was built for {L.T}x{L.K}")
+    if y.shape[0] < L.P_cap or y.shape[1] != H:
+        raise ValueError(f"y must have at least P_cap={L.P_cap} rows of {H}, got "
+                         f"{tuple(y.shape)}")
     if grad_y is None:
         grad_y = torch.empty((L.P_cap, H), dtype=torch.bfloat16, device=y.device)
     if grad_scales is None:
@@ -361,6 +377,10 @@ def moe_dispatch_bwd(grad_xp: torch.Tensor, dst_row: torch.Tensor, T: int, K: in
     _cuda(grad_xp, "grad_xp", torch.bfloat16)
     _cuda(dst_row, "dst_row", torch.int32)
     H = grad_xp.shape[1]
+    if dst_row.numel() < T * K:
+        raise ValueError(f"dst_row has {dst_row.numel()} entries, needs T*K = {T * K}")
+    if P_cap is not None and P_cap > grad_xp.shape[0]:
+        raise ValueError(f"P_cap={P_cap} exceeds the {grad_xp.shape[0]} rows of grad_xp")
     if grad_x is None:
         grad_x = torch.empty((T, H), dtype=torch.bfloat16, device=grad_xp.device)
     _shape(_cuda(grad_x, "grad_x", torch.bfloat16), "grad_x", (T, H))

@@ -54,3 +54,33 @@ def test_every_call_accepts_an_empty_batch(K, E, R, H):
     assert res[0].shape == (0, H)
     torch.cuda.synchronize()
     assert ops.read_status(st) == 0
+
+
+def test_binding_rejects_inconsistent_shapes():
+    """The binding refuses shapes that would make a kernel read or write past
+    a buffer, before anything is launched."""
+    st = ops.new_status()
+    ids = torch.randint(0, 8, (64, 1), dtype=torch.int32, device=DEV)
+    L = ops.moe_dispatch_layout(ids, 8, 2, status=st)
+    x = torch.zeros((65, 128), dtype=torch.bfloat16, device=DEV)          # one row too many
+    with pytest.raises(ValueError):
+        ops.moe_dispatch_permute(x, L)
+    with pytest.raises(ValueError):
+        ops.moe_dispatch_permute_quant(x, L)
+    y = torch.zeros((L.P_cap, 128), dtype=torch.bfloat16, device=DEV)
+    sc = torch.ones((64, 2), dtype=torch.float32, device=DEV)              # K=2 > layout's 1
+    with pytest.raises(ValueError):
+        ops.moe_combine(y, L.dst_row, sc)                                  # dst_row too short
+    with pytest.raises(ValueError):
+        ops.moe_combine(y, L.dst_row, sc[:, :1], P_cap=L.P_cap + 1)        # P_cap past y
+    with pytest.raises(ValueError):
+        ops.moe_combine(y, L.dst_row, sc[:, :1], shared_x=x)               # shared_x rows
+    with pytest.raises(ValueError):
+        ops.moe_dispatch_bwd(y, L.dst_row, 64, 2)                          # dst_row too short
+    g = torch.zeros((64, 128), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ValueError):
+        ops.moe_combine_bwd(g, y[:-1], sc[:, :1], L)                       # y shorter than P_cap
+    with pytest.raises(ValueError):
+        ops.moe_combine_bwd(g, y, sc, L)                                   # K differs from layout
+    torch.cuda.synchronize()
+    assert ops.read_status(st) == 0
