@@ -250,8 +250,10 @@ MOE_API int moe_dispatch_permute_consume(const void* x, int dtype, int64_t T, in
  *   padding rows: code 0x00, scale 0.0f; rows >= P untouched.
  * In:  x bf16 [T, H], row stride x_row_stride elements (multiple of 8),
  *      16-byte aligned; H % 128 == 0.
- * Out: xp uint8 [P_cap, H] (16-byte aligned); xp_scales fp32 [P_cap, H/128];
- *      tile_ready (nullable) as in moe_dispatch_permute.
+ * Out: xp uint8 [P_cap, H] (16-byte aligned); xp_scales fp32 [P_cap, H/128]
+ *      (4-byte aligned; with 16-byte alignment and H % 512 == 0 the scales
+ *      are bulk-stored with the codes); tile_ready (nullable) as in
+ *      moe_dispatch_permute.
  * Data errors: MOE_ERR_BOUNDS as in moe_dispatch_permute.
  */
 MOE_API int moe_dispatch_permute_quant(const void* x, int64_t T, int H, int64_t x_row_stride,
@@ -310,8 +312,10 @@ MOE_API int moe_dispatch_bwd(const void* grad_xp, const int32_t* dst_row, int64_
  *   s = amax|x| / 448 in fp32 (1 if amax == 0);
  *   q = E4M3(x / s) with fp32 division, round-to-nearest-even, saturating
  *       at +-448.
- * In:  x bf16 [T, H], row stride x_row_stride elements; H % 128 == 0.
- * Out: q uint8 [T, H] contiguous; q_scales fp32 [T, H/128] contiguous.
+ * In:  x bf16 [T, H], row stride x_row_stride elements (multiple of 8),
+ *      16-byte aligned; H % 128 == 0.
+ * Out: q uint8 [T, H] contiguous, 8-byte aligned (16-byte aligned q is
+ *      written with 16-byte stores); q_scales fp32 [T, H/128] contiguous.
  */
 MOE_API int moe_quantize_e4m3(const void* x, int64_t T, int H, int64_t x_row_stride, void* q,
                       float* q_scales, int32_t* d_status, void* stream);
