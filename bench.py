@@ -78,6 +78,22 @@ def step_bytes(T, K, H, E, P, fwd_only=False):
     return b
 
 
+def groups_gbs(nbytes, phase_us):
+    """Algorithmic GB/s of dispatch (layout + permute), of combine, of their
+    sum (the forward pass) and, when timed, of the two backward calls, from
+    the per-kernel times."""
+    groups = {"dispatch": ("layout", "permute"), "combine": ("combine",),
+              "dispatch_plus_combine": ("layout", "permute", "combine"),
+              "backward": ("combine_bwd", "dispatch_bwd")}
+    out = {}
+    for g, ps in groups.items():
+        if all(p in phase_us for p in ps):
+            b = sum(nbytes[p] for p in ps)
+            us = sum(phase_us[p] for p in ps)
+            out[g] = {"GBps": round(b / (us * 1e-6) / 1e9, 1), "us": round(us, 2), "bytes": b}
+    return out
+
+
 def measured_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -372,6 +388,7 @@ def run_ours(args, world, rank, local):
                           f"kernels (which serialises them): {phase_step_ms:.4f} ms per step "
                           "there, against ms_per_step in the timed region",
            "phases_gbs": {p: round(v, 1) for p, v in phase_gbs.items()},
+           "groups_gbs": groups_gbs(nbytes, phase_us),
            "roofline": roofline,
            "gpu_launches": LAUNCHES_PER_STEP[args.fwd_only] * args.steps,
            "clocks": clk.summary()}

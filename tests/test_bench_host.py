@@ -98,3 +98,15 @@ def test_bf16_max_ulp_units():
     assert bench.bf16_max_ulp(one, one) == 0.0
     # 2.0 vs 1.0: one unit of 1.0's binade is 2^-7, so the gap is 128 ulps
     assert bench.bf16_max_ulp(np.array([0x4000], np.uint16), one) == 128.0
+
+
+def test_groups_gbs_sums_bytes_and_times():
+    nb = {"layout": 100, "permute": 900, "combine": 500, "combine_bwd": 1000, "dispatch_bwd": 400}
+    us = {"layout": 1.0, "permute": 9.0, "combine": 5.0, "combine_bwd": 10.0, "dispatch_bwd": 4.0}
+    g = bench.groups_gbs(nb, us)
+    assert g["dispatch"] == {"GBps": 0.1, "us": 10.0, "bytes": 1000}
+    assert g["dispatch_plus_combine"]["bytes"] == 1500 and g["dispatch_plus_combine"]["us"] == 15.0
+    assert g["backward"]["bytes"] == 1400
+    fwd = bench.groups_gbs({k: nb[k] for k in ("layout", "permute", "combine")},
+                           {k: us[k] for k in ("layout", "permute", "combine")})
+    assert "backward" not in fwd
