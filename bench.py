@@ -691,16 +691,22 @@ def extra_workloads(args, dev, flush, stream):
         ("permute_quant_fused", lambda: ops.moe_dispatch_permute_quant(x, L, xp=xp,
                                                                        xp_scales=xps)),
         ("combine", lambda: ops.moe_combine(y, L.dst_row, sc, out=out)),
+        # the forward pass as one chained step: layout, fused FP8 dispatch, combine
+        ("fwd_step", lambda: (ops.moe_dispatch_layout(ids, E, R, layout=L),
+                              ops.moe_dispatch_permute_quant(x, L, xp=xp, xp_scales=xps),
+                              ops.moe_combine(y, L.dst_row, sc, out=out))),
     ], flush, steps, stream)
     b = {"layout": 8 * T * K + 4 * P, "quantize": 2 * T * H + T * H + 4 * T * nb,
          "permute_e4m3": T * H + 4 * T * nb + P * H + 4 * P * nb,
          "permute_quant_fused": 2 * T * H + P * H + 4 * P * nb,
          "combine": 2 * T * K * H + 8 * T * K + 2 * T * H}
+    b["fwd_step"] = b["layout"] + b["permute_quant_fused"] + b["combine"]
     res[s.name] = {"T": T, "H": H, "E": E, "K": K, "P": P,
                    "us": {k: round(v, 1) for k, v in t.items()},
                    "GBps": {k: round(b[k] / (t[k] * 1e-6) / 1e9, 1) for k in t},
                    "dispatch_unfused_us": round(t["quantize"] + t["permute_e4m3"], 1),
-                   "dispatch_fused_us": round(t["permute_quant_fused"], 1)}
+                   "dispatch_fused_us": round(t["permute_quant_fused"], 1),
+                   "fwd_step_tokens_per_s": round(T / (t["fwd_step"] * 1e-6), 1)}
     del x, q, qs, xp, xps, y, out, L
     torch.cuda.empty_cache()
 
@@ -721,16 +727,21 @@ def extra_workloads(args, dev, flush, stream):
         ("layout", lambda: ops.moe_dispatch_layout(ids, E, R, layout=L)),
         ("permute", lambda: ops.moe_dispatch_permute(x, L, xp=xp)),
         ("combine_shared", lambda: ops.moe_combine(y, L.dst_row, sc, shared_x=sh, out=out)),
+        ("fwd_step", lambda: (ops.moe_dispatch_layout(ids, E, R, layout=L),
+                              ops.moe_dispatch_permute(x, L, xp=xp),
+                              ops.moe_combine(y, L.dst_row, sc, shared_x=sh, out=out))),
     ], flush, steps, stream)
     b = {"layout": 8 * T * K + 4 * P, "permute": 2 * T * H + 2 * P * H,
          "combine_shared": 2 * T * K * H + 8 * T * K + 4 * T * H}
+    b["fwd_step"] = b["layout"] + b["permute"] + b["combine_shared"]
     res[s.name] = {"T": T, "H": H, "E": E, "K": K, "P": P,
                    "us": {k: round(v, 1) for k, v in t.items()},
                    "GBps": {k: round(b[k] / (t[k] * 1e-6) / 1e9, 1) for k in t}}
     del x, xp, y, sh, out, L
     torch.cuda.empty_cache()
 
-    # backward under skew: the hot expert in 60% of the rows, and the stress variant with it in every row
+    # backward under skew: the hot expert in 60% of the rows, and the stress
+    # variant with it in every row
     for name, spec in (("bwd_skew", W.config(5)),
                        ("bwd_skew_hot100", W.config(5).with_(hot_p=1.0))):
         s = spec
@@ -749,10 +760,13 @@ def extra_workloads(args, dev, flush, stream):
             ("layout", lambda: ops.moe_dispatch_layout(ids, E, R, layout=L)),
             ("combine_bwd", lambda: ops.moe_combine_bwd(g, y, sc, L, grad_y=gy, grad_scales=gs)),
             ("dispatch_bwd", lambda: ops.moe_dispatch_bwd(gy, L.dst_row, T, K, grad_x=gx)),
+            ("bwd_step", lambda: (ops.moe_combine_bwd(g, y, sc, L, grad_y=gy, grad_scales=gs),
+                                  ops.moe_dispatch_bwd(gy, L.dst_row, T, K, grad_x=gx))),
         ], flush, steps, stream)
         b = {"layout": 8 * T * K + 4 * P,
              "combine_bwd": 2 * T * H + 2 * T * K * H + 2 * P * H + 12 * T * K,
              "dispatch_bwd": 2 * T * K * H + 2 * T * H + 4 * T * K}
+        b["bwd_step"] = b["combine_bwd"] + b["dispatch_bwd"]
         res[name] = {"T": T, "H": H, "E": E, "K": K, "P": P, "hot_p": s.hot_p,
                      "us": {k: round(v, 1) for k, v in t.items()},
                      "GBps": {k: round(b[k] / (t[k] * 1e-6) / 1e9, 1) for k in t}}
