@@ -146,7 +146,7 @@ constexpr int kBwdThreads = MOE_BWD_THREADS;
 constexpr int kBwdWarps = kBwdThreads / 32;
 
 // resident CTAs per SM asked of the register allocator, per column batch
-constexpr int bwd_min_blocks(int u) { return u == 1 ? 5 : u == 2 ? 4 : 3; }
+constexpr int bwd_min_blocks(int u) { return u == 8 ? 3 : u == 1 ? 5 : 4; }
 
 template <int kU>
 __global__ void __launch_bounds__(kBwdThreads, bwd_min_blocks(kU))
