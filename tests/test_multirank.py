@@ -70,3 +70,14 @@ def test_reference_arm_under_two_ranks_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "GB/s"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    # the same metric, workload and direction as the library's own line
+    assert d["metric"] == bench_metric() and d["higher_is_better"] is True
+    assert d["config"]["workload"].startswith("dsv3_decode: T=4096 H=7168 E=256 K=8 R=8")
+    assert d["steps"] == 1 and d["warmup"] == 1
+    assert d["e2e"]["value"] == d["value"] == d["cpu_baseline"]["value"]
+
+
+def bench_metric():
+    sys.path.insert(0, ROOT)
+    import bench
+    return bench.METRIC
