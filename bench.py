@@ -10,7 +10,9 @@ ranks, Zipf(0.6) routing):
     (identity experts: y = the dispatched rows) -> combine backward ->
     dispatch backward.
 value = algorithmic HBM bytes of the step / device time of the step, in GB/s
-(also reported: tokens/s).  Inputs are resident in HBM when the timed region
+(also reported: tokens/s).  fwd_step times the forward pair alone (layout ->
+permute -> combine: dispatch + combine, the metric's pair) the same way over
+the same number of steps.  Inputs are resident in HBM when the timed region
 starts; L2 is flushed (256 MiB write) before every timed step and the flush
 is outside the timed events.  Inside the timed region the only events are
 one before and one after each step; per-kernel times (phases_us, and the
@@ -302,27 +304,37 @@ def run_ours(args, world, rank, local):
     # Timed region: one event before and one after each step, none between
     # the kernels (an event between two kernels ends the programmatic launch
     # chain and serialises them: ~5 us per boundary).
-    bounds = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(smi_id(torch, dev)) as clk:
+    def timed_steps(fn):
+        bounds = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize()
         for i in range(args.steps):
             flush.zero_()
             bounds[i][0].record(stream)
-            if graph is not None:
-                graph.replay()
-            else:
-                step()
+            fn()
             bounds[i][1].record(stream)
         torch.cuda.synchronize()
-    barrier(world)
-    step_ms = [a.elapsed_time(b) for a, b in bounds]
+        barrier(world)
+        return [a.elapsed_time(b) for a, b in bounds]
+
+    def forward():  # dispatch + combine: the metric's pair, chained
+        ops.moe_dispatch_layout(ids, E, R, layout=L, status=st)
+        ops.moe_dispatch_permute(x, L, xp=xp, status=st)
+        ops.moe_combine(xp, L.dst_row, sc, out=out, status=st)
+
+    with ClockSampler(smi_id(torch, dev)) as clk:
+        step_ms = timed_steps(graph.replay if graph is not None else step)
+        # The forward step alone (layout -> permute -> combine), timed the same
+        # way over the same number of steps; with --fwd-only it is the step.
+        fwd_ms = step_ms if args.fwd_only else timed_steps(forward)
+    if ops.read_status(st) != 0:
+        raise RuntimeError(f"device status {ops.read_status(st)} in the timed steps")
     snapshot = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # the last timed step's outputs, checked against the oracle's pass in
         # the cpu_baseline leg
-        snapshot = {"counts": L.expert_counts, "offsets": L.expert_offsets,
+        snapshot = {"counts": L.expert_counts, "offsets": L.expert_offsets, "scales": sc,
                     "rank_counts": L.rank_counts, "rank_offsets": L.rank_offsets,
                     "dst_row": L.dst_row, "row_src": L.row_src, "out": out.view(torch.int16)}
         if not args.fwd_only:
@@ -357,8 +369,17 @@ def run_ours(args, world, rank, local):
     phase_gbs = {p: nbytes[p] / (phase_us[p] * 1e-6) / 1e9 for p in phases}
     dom = max((p for p in phases if p != "layout"), key=lambda p: phase_us[p])
     peak, peak_src = measured_peak()
-    fwd_us = sum(phase_us[p] for p in ("layout", "permute", "combine"))
     fwd_bytes = sum(nbytes[p] for p in ("layout", "permute", "combine"))
+    fwd_ms_per_step = max_over_ranks(sum(fwd_ms), world) / args.steps
+    fwd_gbs = fwd_bytes * world / (fwd_ms_per_step * 1e-3) / 1e9
+    fwd_step = {"ms": round(fwd_ms_per_step, 5), "GBps": round(fwd_gbs, 1),
+                "frac": round(fwd_gbs / world / peak, 4),
+                "tokens_per_s": round(T * world / (fwd_ms_per_step * 1e-3), 1),
+                "bytes": fwd_bytes, "steps": args.steps,
+                "median_ms": round(statistics.median(fwd_ms), 5),
+                "what": "layout -> permute -> combine chained on one stream, no events between "
+                        "the kernels, L2 flushed before each step (outside the events); max "
+                        "over ranks"}
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(phase_gbs[dom], 1),
                 "peak": peak, "unit": "GB/s", "frac": round(phase_gbs[dom] / peak, 4),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src ==
@@ -369,7 +390,7 @@ def run_ours(args, world, rank, local):
                                    "the timed region (events on the launching stream on both "
                                    "sides of each kernel, L2 flushed before each step)",
                 "step_frac": round(bytes_step / (ms_per_step * 1e-3) / 1e9 / peak, 4),
-                "fwd_frac": round(fwd_bytes / (fwd_us * 1e-6) / 1e9 / peak, 4)}
+                "fwd_step_frac": fwd_step["frac"]}
 
     res = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s",
            "tokens_per_s": round(tok_s, 1), "n_gpus": world, "steps": args.steps,
@@ -390,7 +411,9 @@ def run_ours(args, world, rank, local):
            "phases_gbs": {p: round(v, 1) for p, v in phase_gbs.items()},
            "groups_gbs": groups_gbs(nbytes, phase_us),
            "roofline": roofline,
-           "gpu_launches": LAUNCHES_PER_STEP[args.fwd_only] * args.steps,
+           "fwd_step": fwd_step,
+           "gpu_launches": LAUNCHES_PER_STEP[args.fwd_only] * args.steps +
+           (0 if args.fwd_only else LAUNCHES_PER_STEP[True] * args.steps),
            "clocks": clk.summary()}
     if snapshot is not None:
         res["_timed_outputs"] = snapshot
@@ -737,6 +760,12 @@ def extra_workloads(args, dev, flush, stream):
     res[s.name] = {"T": T, "H": H, "E": E, "K": K, "P": P,
                    "us": {k: round(v, 1) for k, v in t.items()},
                    "GBps": {k: round(b[k] / (t[k] * 1e-6) / 1e9, 1) for k in t}}
+    if not args.no_cpu_baseline:
+        # the last timed combine's output and its inputs, for the check of its
+        # elements against the exact sum (done on the host after the GPU work)
+        res[s.name]["_combine_snapshot"] = {
+            "out": W.as_u16(out.cpu()), "y": W.as_u16(y.cpu()), "dst_row": L.dst_row.cpu().numpy(),
+            "scales": sc.cpu().numpy(), "shared": W.as_u16(sh.cpu())}
     del x, xp, y, sh, out, L
     torch.cuda.empty_cache()
 
@@ -900,6 +929,41 @@ def bf16_max_ulp(gpu_bits, ref_bits):
     return float(np.max(np.abs(g - r) / ulp)) if g.size else 0.0
 
 
+def combine_exceptions(out_bits, y_bits, dst_row, scales, shared_bits=None, chunk=256):
+    """Elements of a combine output farther than one bf16 ulp (2^-7 |exact|)
+    from the exact sum (fp64), and how many of those are NOT cancellation
+    cases.  An fp32 running sum of n terms is within gamma_n * sum|terms| of
+    the exact sum, and rounding it once to bf16 adds at most 2^-8 of its
+    magnitude, so an element can pass one ulp only where
+    |exact| < 257 * gamma_n * sum|terms| (n = K, plus one with a shared
+    term): those are the cancellation cases; any other exception is a bug."""
+    import numpy as np
+
+    def f(b):
+        return (np.asarray(b).view(np.uint16).astype(np.uint32) << 16).view(np.float32) \
+            .astype(np.float64)
+    T, K = scales.shape
+    n = K + (0 if shared_bits is None else 1)
+    gam = n * 2.0 ** -24 / (1 - n * 2.0 ** -24)
+    rows = np.asarray(dst_row)[:T * K].reshape(T, K)
+    over = not_cancel = 0
+    for a in range(0, T, chunk):
+        b = min(T, a + chunk)
+        yv = f(y_bits[rows[a:b]])                              # [c, K, H]
+        sv = scales[a:b].astype(np.float64)
+        exact = np.einsum("tk,tkh->th", sv, yv)
+        mag = np.einsum("tk,tkh->th", np.abs(sv), np.abs(yv))
+        if shared_bits is not None:
+            sh = f(shared_bits[a:b])
+            exact += sh
+            mag += np.abs(sh)
+        o = np.abs(f(out_bits[a:b]) - exact) > 2.0 ** -7 * np.abs(exact)
+        over += int(o.sum())
+        not_cancel += int((o & (np.abs(exact) >= 257 * gam * mag + 2.0 ** -126)).sum())
+    return {"elements": int(T * y_bits.shape[1]), "over_one_ulp_of_exact": over,
+            "over_one_ulp_not_cancellation": not_cancel}
+
+
 def check_timed_outputs(s, res, gpu, x, g, fwd_only):
     """The last timed GPU step against the oracle's pass over the same inputs:
     integers and the permuted bytes must be identical; the bf16 outputs are
@@ -919,9 +983,13 @@ def check_timed_outputs(s, res, gpu, x, g, fwd_only):
     chk["permute_bytes_exact"] = bool(gpu["xp"].shape[0] == P and np.array_equal(
         gpu["xp"].view(np.uint16), res["xp"][:P]))
     chk["combine_max_ulp"] = round(bf16_max_ulp(gpu["out"], res["out"]), 3)
+    chk["combine_vs_exact_sum"] = combine_exceptions(gpu["out"], res["xp"], L.dst_row,
+                                                     gpu["scales"])
     if not fwd_only:
         chk["combine_bwd_grad_y_max_ulp"] = round(
             bf16_max_ulp(gpu["grad_y"], res["grad_y"][:P]), 3)
+        chk["combine_bwd_grad_y_bit_exact"] = bool(np.array_equal(
+            gpu["grad_y"].view(np.uint16), res["grad_y"][:P]))
         chk["dispatch_bwd_max_ulp"] = round(bf16_max_ulp(gpu["grad_x"], res["grad_x"]), 3)
 
         def f(b):
@@ -1032,10 +1100,17 @@ def main():
     try:
         res = run_ours(args, world, rank, local)
         timed = res.pop("_timed_outputs", None)
+        shared_snap = res.get("other_workloads", {}).get("shared_expert", {}).pop(
+            "_combine_snapshot", None)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(args.fwd_only)
             res["cpu_baseline_all_cores"], res["timed_run_check"] = \
                 cpu_baseline_all_cores(args.fwd_only, timed)
+            if shared_snap is not None:
+                res["timed_run_check"]["shared_expert_combine_vs_exact_sum"] = \
+                    combine_exceptions(shared_snap["out"], shared_snap["y"],
+                                       shared_snap["dst_row"], shared_snap["scales"],
+                                       shared_snap["shared"])
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -20,7 +20,8 @@
 //     fp32 reduction runs k = 0..K-1 in order with fma, then adds the shared
 //     row, then rounds once.
 //   * combine_bwd: a 128-thread CTA owns a token row: it reads grad_out[t]
-//     once, gathers the K rows of y, writes the K scaled rows of grad_y and
+//     once, gathers the K rows of y, writes the K scaled rows of grad_y
+//     (each element the exact product rounded once to bf16) and
 //     reduces the K dot products across the CTA in a fixed order
 //     (deterministic).  The same CTAs then zero the padding rows of grad_y.
 #include "common.cuh"
@@ -139,6 +140,26 @@ gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restri
   }
 }
 
+// s * g as an fp32 value whose round-to-nearest-even bf16 conversion equals
+// the conversion of the exact product (one rounding, as the definition of
+// grad_y asks).  The fp32 product p = RN32(s * g) is rounded the same way as
+// the exact product unless p sits exactly on a midpoint between two bf16
+// values (low 16 bits 0x8000): RN32 is monotone and every bf16 midpoint is an
+// fp32 value, so otherwise p and the exact product lie on the same side of
+// every midpoint.  On a midpoint reached by rounding, the exact product
+// (24 + 8 significant bits, so exact in fp64) tells on which side it lies
+// and p moves one fp32 ulp toward it, off the tie.  For random data this
+// branch is taken about once in 65536 products.
+__device__ __forceinline__ float scaled_for_bf16(float s, float g) {
+  const float p = __fmul_rn(s, g);
+  const uint32_t b = __float_as_uint(p);
+  if ((b & 0xFFFFu) != 0x8000u) return p;
+  const double v = (double)s * (double)g;
+  const double pd = (double)p;
+  if (v == pd) return p;
+  return __uint_as_float(fabs(v) > fabs(pd) ? b + 1u : b - 1u);
+}
+
 #ifndef MOE_BWD_THREADS
 #define MOE_BWD_THREADS 128
 #endif
@@ -238,10 +259,10 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
               d = fmaf(gf[i][2 * q + 1], bf16_hi(yw[q]), d);
             }
             uint4 o;
-            o.x = pack_bf16x2(__fmul_rn(sk, gf[i][0]), __fmul_rn(sk, gf[i][1]));
-            o.y = pack_bf16x2(__fmul_rn(sk, gf[i][2]), __fmul_rn(sk, gf[i][3]));
-            o.z = pack_bf16x2(__fmul_rn(sk, gf[i][4]), __fmul_rn(sk, gf[i][5]));
-            o.w = pack_bf16x2(__fmul_rn(sk, gf[i][6]), __fmul_rn(sk, gf[i][7]));
+            o.x = pack_bf16x2(scaled_for_bf16(sk, gf[i][0]), scaled_for_bf16(sk, gf[i][1]));
+            o.y = pack_bf16x2(scaled_for_bf16(sk, gf[i][2]), scaled_for_bf16(sk, gf[i][3]));
+            o.z = pack_bf16x2(scaled_for_bf16(sk, gf[i][4]), scaled_for_bf16(sk, gf[i][5]));
+            o.w = pack_bf16x2(scaled_for_bf16(sk, gf[i][6]), scaled_for_bf16(sk, gf[i][7]));
             st_v4(grad_y + (int64_t)r * H + (int64_t)vec * 8, o);
           }
           dot[k] = d;

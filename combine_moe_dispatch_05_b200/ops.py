@@ -157,14 +157,15 @@ class Layout:
     dst_row: torch.Tensor
     row_src: Optional[torch.Tensor]
     tile_ready: Optional[torch.Tensor]
-    workspace: torch.Tensor
+    workspace: Optional[torch.Tensor]   # None for layouts filled by moe_dispatch_layout_static
 
 
 def alloc_layout(T: int, K: int, E: int, R: int, device, P_cap: Optional[int] = None,
-                 with_row_src=True, with_counters=True) -> Layout:
+                 with_row_src=True, with_counters=True, with_workspace=True) -> Layout:
     P_cap = padded_capacity(T, K, E) if P_cap is None else P_cap
     i32 = dict(dtype=torch.int32, device=device)
-    ws = torch.empty(max(1, layout_workspace_bytes(T, K, E)), dtype=torch.uint8, device=device)
+    ws = torch.empty(max(1, layout_workspace_bytes(T, K, E)), dtype=torch.uint8,
+                     device=device) if with_workspace else None
     return Layout(
         T, K, E, R, P_cap,
         torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R, **i32),
@@ -181,6 +182,8 @@ def moe_dispatch_layout(topk_idx: torch.Tensor, E: int, R: int, layout: Optional
     _cuda(topk_idx, "topk_idx", torch.int32)
     T, K = topk_idx.shape
     L = layout or alloc_layout(T, K, E, R, topk_idx.device, P_cap)
+    if L.workspace is None:
+        raise ValueError("this layout has no workspace (use moe_dispatch_layout_static)")
     rc = lib().moe_dispatch_layout(
         _ptr(topk_idx), T, K, E, R, _ptr(L.expert_counts), _ptr(L.expert_offsets),
         _ptr(L.rank_counts), _ptr(L.rank_offsets), _ptr(L.dst_row), _ptr(L.row_src),
@@ -196,11 +199,13 @@ def moe_dispatch_layout_static(topk_idx: torch.Tensor, E: int, R: int,
                                P_cap: Optional[int] = None, stream=None) -> Layout:
     """moe_dispatch_layout without a workspace, for callers that cannot
     allocate device memory at call time: the library's own static scratch is
-    used.  Outputs are still the caller's (pass ``layout`` to avoid any
-    allocation here as well)."""
+    used.  Outputs are still the caller's: pass ``layout`` (for instance from
+    ``alloc_layout(..., with_workspace=False)`` at start-up) so that this call
+    allocates nothing; without it the output tensors, and only those, are
+    allocated here."""
     _cuda(topk_idx, "topk_idx", torch.int32)
     T, K = topk_idx.shape
-    L = layout or alloc_layout(T, K, E, R, topk_idx.device, P_cap)
+    L = layout or alloc_layout(T, K, E, R, topk_idx.device, P_cap, with_workspace=False)
     rc = lib().moe_dispatch_layout_static(
         _ptr(topk_idx), T, K, E, R, _ptr(L.expert_counts), _ptr(L.expert_offsets),
         _ptr(L.rank_counts), _ptr(L.rank_offsets), _ptr(L.dst_row), _ptr(L.row_src),

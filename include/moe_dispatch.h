@@ -46,6 +46,15 @@
  *     the offending writes instead of trapping.  Read it after the stream
  *     has been synchronised.  Outputs are unspecified (but every write stays
  *     inside the buffers) when it is non-zero.
+ *   - After MOE_ERR_TIMEOUT (a device-side wait gave up after its bound) the
+ *     call's outputs are undefined, and so is the device state it leaves:
+ *     a kernel that gave up waits, again bounded, for the copies it issued
+ *     and then exits, and a bulk load that has still not landed by then may
+ *     complete later into shared memory that a later CTA on that SM owns.
+ *     A timeout means the GPU stalled for seconds; the caller should
+ *     synchronise the device, treat every output of the calls since the
+ *     status was last clear as garbage, and re-run them (or restart the
+ *     process, if the stall recurs).
  */
 #ifndef MOE_DISPATCH_H_
 #define MOE_DISPATCH_H_
@@ -156,7 +165,10 @@ MOE_API int moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int K, int E
  *   - Set-up: the first call on each device looks up that device's address
  *     of the array (cudaGetSymbolAddress, with the device current); make
  *     that first call before any stream capture.  A failed lookup returns
- *     MOE_ERR_CUDA.
+ *     MOE_ERR_CUDA.  The address is kept for the life of the process, so a
+ *     device reset (cudaDeviceReset, or anything that destroys the primary
+ *     context) between calls is not supported: the array may move and the
+ *     kept address would then be stale.
  *   - Sharing: all calls on a device use the same array, which keeps the last
  *     call's contents.  Nothing in it needs to start at zero (every word the
  *     kernels read is written earlier in the same call), but calls that may
@@ -195,7 +207,8 @@ MOE_API int moe_dispatch_layout_static(const int32_t* topk_idx, int64_t T, int K
  *            tile whose counter reads 128 with an ld.acquire.gpu is complete.
  * Data errors: MOE_ERR_BOUNDS if a dst_row entry or offset leaves
  *   [0, P_cap) (that write is skipped); MOE_ERR_TIMEOUT if a staged load
- *   did not land within about 2 s.
+ *   did not land within about 2 s (outputs and device state are then
+ *   undefined: see the conventions above).
  */
 MOE_API int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H, int64_t x_row_stride,
                          const float* x_scales, int64_t x_scales_row_stride,

@@ -62,6 +62,7 @@ def test_host_cpu_reports_threads_and_model():
 def _fake_gpu_outputs(s, res):
     L = res["layout"]
     return {"counts": L.counts.copy(), "offsets": L.offsets.copy(),
+            "scales": W.topk_scales(s).numpy(),
             "rank_counts": L.rank_counts.copy(), "rank_offsets": L.rank_offsets.copy(),
             "dst_row": L.dst_row.copy(), "row_src": L.row_src.copy(),
             "xp": res["xp"][:L.P].view(np.int16).copy(), "out": res["out"].view(np.int16).copy(),
@@ -78,18 +79,28 @@ def test_timed_run_check_accepts_identical_and_flags_changes():
     assert ok["layout_bit_exact"] and ok["permute_bytes_exact"]
     assert ok["combine_max_ulp"] == 0 and ok["dispatch_bwd_max_ulp"] == 0
     assert ok["combine_bwd_grad_y_max_ulp"] == 0 and ok["grad_scales_max_err_over_norms"] == 0
+    assert ok["combine_bwd_grad_y_bit_exact"]
+    assert ok["combine_vs_exact_sum"]["over_one_ulp_of_exact"] == 0
+    assert ok["combine_vs_exact_sum"]["elements"] == s.T * s.H
 
     bad = _fake_gpu_outputs(s, res)
     bad["dst_row"][7] += 1
     bad["xp"][3, 5] ^= 1
-    bad["out"][2, 9] += 1          # one bf16 ulp (same binade)
+    flat = bad["out"].reshape(-1)  # two bf16 ulps (same binade), away from cancellation
+    j = int(np.flatnonzero(((flat.view(np.uint16) & 0x7F) < 0x70) &
+                           ((flat.view(np.uint16) & 0x7F80) > 0x3C00))[0])
+    flat[j] += 2
+    bad["grad_y"][1, 2] ^= 1
     # three ulps, at an element whose mantissa leaves room inside its binade
     flat = bad["grad_x"].reshape(-1)
     i = int(np.flatnonzero((flat.view(np.uint16) & 0x7F) < 0x70)[0])
     flat[i] += 3
     chk = bench.check_timed_outputs(s, res, bad, x, g, False)
     assert not chk["layout_bit_exact"] and not chk["permute_bytes_exact"]
-    assert chk["combine_max_ulp"] == 1 and chk["dispatch_bwd_max_ulp"] == 3
+    assert chk["combine_max_ulp"] == 2 and chk["dispatch_bwd_max_ulp"] == 3
+    assert chk["combine_vs_exact_sum"]["over_one_ulp_of_exact"] == 1
+    assert chk["combine_vs_exact_sum"]["over_one_ulp_not_cancellation"] == 1
+    assert not chk["combine_bwd_grad_y_bit_exact"]
 
 
 def test_bf16_max_ulp_units():

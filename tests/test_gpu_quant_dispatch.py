@@ -90,8 +90,10 @@ def test_fused_equals_unfused_gpu_path_full_prefill():
     assert np.all(cnt[:P // 128] == 128) and np.all(cnt[P // 128:] == 0)
     assert torch.equal(xp1[:P], xp2[:P])
     assert torch.equal(xs1[:P].view(torch.int32), xs2[:P].view(torch.int32))
-    # and sampled tokens against the oracle quantiser
-    rows = torch.randperm(s.T, generator=torch.Generator().manual_seed(1))[:64]
-    q_ref, s_ref = oracle.quantize_e4m3(W.as_u16(x[rows].cpu()))
-    assert np.array_equal(q[rows].cpu().numpy(), q_ref)
-    assert np.array_equal(qs[rows].cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+def test_fused_quant_dispatch_full_prefill_matches_oracle():
+    """Full prefill size (T=32768, H=7168, E=256, K=8, Zipf 1.2): every code
+    and scale of the expert-major buffer, padding rows and the untouched rows
+    past P included, against the oracle's quantiser followed by its permute."""
+    run(W.config(3))

@@ -117,6 +117,56 @@ def test_combine_bwd_grad_scales_and_grad_y():
     assert np.all(gy[L.P:] == 0x7777)
 
 
+def _bf16_nearest_rational(q):
+    """bf16 bits of the value nearest the rational q, ties to the even code
+    (normal range only): exact arithmetic, no floating point."""
+    from fractions import Fraction
+    sign = 0x8000 if q < 0 else 0
+    a = abs(Fraction(q))
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = Fraction(2) ** (e - 7)
+    n = a / ulp                                      # in [128, 256)
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    bits = int(np.float32(float(fl * ulp)).view(np.uint32)) >> 16
+    return sign | bits
+
+
+def test_combine_bwd_grad_y_single_rounding_on_midpoint_products():
+    """grad_y = bf16(s * g) rounded once from the exact product.  On inputs
+    whose fp32 products are bf16 midpoints (tests/_ties.py) the oracle must
+    match an exact rational rounding, and rounding the fp32 product again (a
+    plausible mistake) must differ from it on many elements."""
+    from fractions import Fraction
+
+    from _ties import fraction_on_midpoints, midpoint_products
+    T, K, H, E = 6, 2, 40, 4
+    sc, gf = midpoint_products(T, K, H, seed=12)
+    assert fraction_on_midpoints(sc, gf) > 0.3
+    g = (gf.view(np.uint32) >> 16).astype(np.uint16)          # exact: gf holds bf16 values
+    ids = np.array([[t % E, (t + 1) % E] for t in range(T)], np.int32)
+    L = oracle.layout(ids, E, 1)
+    y = np.zeros((L.P_cap, H), np.uint16)
+    gy = np.zeros((L.P_cap, H), np.uint16)
+    oracle.combine_bwd(g, y, sc, L.dst_row, L.counts, L.offsets, gy)
+    rows = L.dst_row.reshape(T, K)
+    twice = W.as_u16(torch.from_numpy(sc[:, :, None] * gf[:, None, :]).to(torch.bfloat16))
+    differ = 0
+    for t in range(T):
+        for k in range(K):
+            for h in range(H):
+                want = _bf16_nearest_rational(Fraction(float(sc[t, k])) * Fraction(float(gf[t, h])))
+                assert gy[rows[t, k], h] == want, (t, k, h)
+                differ += int(twice[t, k, h] != want)
+    assert differ > 0.1 * T * K * H
+
+
 def test_combine_bwd_adjoint_identity():
     """<combine(y), g> == <y, grad_y> and d<combine, g>/ds = grad_s (linearity)."""
     s, ids, L, y, sc, _ = setup(40, 4, 6, 48, 9)

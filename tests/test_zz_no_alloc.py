@@ -59,11 +59,57 @@ def test_static_layout_matches_workspace_layout_on_consecutive_calls():
         assert _call_static(ids, s.E, s.R, o) == ops.OK
         torch.cuda.synchronize()
         assert ops.read_status(ref_status) == 0 and int(o["status"].item()) == 0
-        for mine, theirs in [("counts", ref.expert_counts), ("offsets", ref.expert_offsets),
-                             ("rank_counts", ref.rank_counts), ("rank_offsets", ref.rank_offsets),
-                             ("dst_row", ref.dst_row), ("row_src", ref.row_src),
-                             ("tile_ready", ref.tile_ready)]:
-            assert torch.equal(o[mine], theirs), (s.name, mine)
+        _assert_same(o, ref, s.name)
+
+
+def _assert_same(o, ref, what):
+    for mine, theirs in [("counts", ref.expert_counts), ("offsets", ref.expert_offsets),
+                         ("rank_counts", ref.rank_counts), ("rank_offsets", ref.rank_offsets),
+                         ("dst_row", ref.dst_row), ("row_src", ref.row_src),
+                         ("tile_ready", ref.tile_ready)]:
+        assert torch.equal(o[mine], theirs), (what, mine)
+
+
+@pytest.mark.gpu
+def test_static_layout_at_the_largest_accepted_size():
+    """T = 116480, K = 8, E = 256: the largest size whose scratch fits the
+    4 MiB array (455 count blocks fill 4193280 of its 4194304 bytes), so the
+    end of the array is written and read back; ids are distinct per row and
+    drawn at random.  Two calls in a row, each equal to the workspace form."""
+    ensure_lib()
+    T, K, E, R = 116480, 8, 256, 8
+    assert ops.layout_workspace_bytes(T, K, E) == 4193280
+    for seed in (5, 6):
+        s = W.Spec("max", T, 64, E, K, R, "uniform", seed=seed)
+        ids = W.topk_ids(s).to(DEV)
+        ref_status = ops.new_status()
+        ref = ops.moe_dispatch_layout(ids, E, R, status=ref_status)
+        o = _outputs(T, K, E, R)
+        assert _call_static(ids, E, R, o) == ops.OK
+        torch.cuda.synchronize()
+        assert ops.read_status(ref_status) == 0 and int(o["status"].item()) == 0
+        _assert_same(o, ref, f"T={T} seed={seed}")
+
+
+@pytest.mark.gpu
+def test_static_layout_through_the_binding_allocates_no_workspace():
+    """ops.moe_dispatch_layout_static with outputs from
+    alloc_layout(with_workspace=False): no workspace tensor exists, and the
+    result equals the workspace form's."""
+    ensure_lib()
+    s = W.config(2)
+    ids = W.topk_ids(s).to(DEV)
+    ref = ops.moe_dispatch_layout(ids, s.E, s.R)
+    L = ops.alloc_layout(s.T, s.K, s.E, s.R, DEV, with_workspace=False)
+    assert L.workspace is None
+    st = ops.new_status()
+    got = ops.moe_dispatch_layout_static(ids, s.E, s.R, layout=L, status=st)
+    assert got is L and ops.read_status(st) == 0
+    o = dict(counts=L.expert_counts, offsets=L.expert_offsets, rank_counts=L.rank_counts,
+             rank_offsets=L.rank_offsets, dst_row=L.dst_row, row_src=L.row_src,
+             tile_ready=L.tile_ready)
+    _assert_same(o, ref, "binding")
+    assert ops.moe_dispatch_layout_static(ids, s.E, s.R).workspace is None
 
 
 @pytest.mark.gpu
