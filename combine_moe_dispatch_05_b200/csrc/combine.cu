@@ -148,8 +148,9 @@ gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restri
 // fp32 value, so otherwise p and the exact product lie on the same side of
 // every midpoint.  On a midpoint reached by rounding, the exact product
 // (24 + 8 significant bits, so exact in fp64) tells on which side it lies
-// and p moves one fp32 ulp toward it, off the tie.  For random data this
-// branch is taken about once in 65536 products.
+// and p moves one fp32 ulp toward it, off the tie.  The caller tests eight
+// products at once and calls this only for a vector that holds a midpoint
+// (for random data about one vector in 8192).
 __device__ __forceinline__ float scaled_for_bf16(float s, float g) {
   const float p = __fmul_rn(s, g);
   const uint32_t b = __float_as_uint(p);
@@ -258,11 +259,22 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
               d = fmaf(gf[i][2 * q], bf16_lo(yw[q]), d);
               d = fmaf(gf[i][2 * q + 1], bf16_hi(yw[q]), d);
             }
+            float pr[8];
+            bool tie = false;  // an fp32 product on a bf16 midpoint: about 1 vector in 8192
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              pr[q] = __fmul_rn(sk, gf[i][q]);
+              tie |= (__float_as_uint(pr[q]) & 0xFFFFu) == 0x8000u;
+            }
+            if (tie) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) pr[q] = scaled_for_bf16(sk, gf[i][q]);
+            }
             uint4 o;
-            o.x = pack_bf16x2(scaled_for_bf16(sk, gf[i][0]), scaled_for_bf16(sk, gf[i][1]));
-            o.y = pack_bf16x2(scaled_for_bf16(sk, gf[i][2]), scaled_for_bf16(sk, gf[i][3]));
-            o.z = pack_bf16x2(scaled_for_bf16(sk, gf[i][4]), scaled_for_bf16(sk, gf[i][5]));
-            o.w = pack_bf16x2(scaled_for_bf16(sk, gf[i][6]), scaled_for_bf16(sk, gf[i][7]));
+            o.x = pack_bf16x2(pr[0], pr[1]);
+            o.y = pack_bf16x2(pr[2], pr[3]);
+            o.z = pack_bf16x2(pr[4], pr[5]);
+            o.w = pack_bf16x2(pr[6], pr[7]);
             st_v4(grad_y + (int64_t)r * H + (int64_t)vec * 8, o);
           }
           dot[k] = d;

@@ -27,6 +27,8 @@
 //     request's atom.acq_rel.gpu on every add is a full fence per row).  FP8
 //     scale rows are copied by the 32 lanes with plain stores before the
 //     same release.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -36,7 +38,10 @@ namespace {
 #define MOE_PERM_MAX_CHUNK 16384
 #endif
 #ifndef MOE_PERM_REL_LAG
-#define MOE_PERM_REL_LAG 2
+#define MOE_PERM_REL_LAG 4
+#endif
+#ifndef MOE_PERM_REL_BATCH
+#define MOE_PERM_REL_BATCH 8
 #endif
 #ifndef MOE_PERM_CTAS_PER_SM
 #define MOE_PERM_CTAS_PER_SM 0  // 0: chosen from the row size
@@ -78,6 +83,10 @@ struct PermArgs {
   uint32_t stage_bytes; // chunk_cap rounded up to 128
   int n_chunks;
   int stages;
+  uint32_t* work;            // [2] claim counter and done count (token-ordered pipeline)
+  int64_t tokens_per_ticket; // tokens named by one token ticket
+  int64_t pad_per_ticket;    // padding rows named by one padding ticket
+  int first_tickets;         // tickets each CTA claims at once to fill its ring
 };
 
 __device__ __forceinline__ uint32_t chunk_len(const PermArgs& a, int ch) {
@@ -85,108 +94,129 @@ __device__ __forceinline__ uint32_t chunk_len(const PermArgs& a, int ch) {
   return (uint32_t)(rem < (int64_t)a.chunk_cap ? rem : (int64_t)a.chunk_cap);
 }
 
-// Destination row of a slot, or -1 if it must be skipped (unplaced slot, or a
-// row outside the buffer, which is reported).
-__device__ __forceinline__ int64_t checked_row(const PermArgs& a, int64_t slot) {
-  const int32_t r = __ldg(a.dst_row + slot);
-  if (r == -1) return -1;
-  if (r < 0 || (int64_t)r >= a.P_cap) {
-    record_error(a.status, MOE_ERR_BOUNDS);
-    return -1;
-  }
-  return r;
-}
+// ---------------------------------------------------------------------------
+// Token-ordered copy pipeline with dynamic work claiming.
+//
+// Work is handed out as tickets: tickets [0, n_tok) each name tpt
+// consecutive tokens, tickets [n_tok, n_tok + n_pad) each name ppt
+// consecutive padding rows (in padding-index order).  CTA c starts with the
+// fixed batch [c*b, c*b + b) (b = enough tokens to fill its ring), so its
+// first loads need no atomic; every later ticket comes from one claim
+// counter (work[0]: ticket G*b + the counter's old value), taken whenever the
+// ring needs another token.  CTAs on faster SMs simply take more tickets, so
+// all of them finish together; the padding tickets come last and fill the
+// tail with load-free stores.  (With equal static shares the CTAs' finishing
+// times spread over ~30 us of a ~135 us launch.)  A second word (work[1])
+// counts CTAs that are done; the last one returns both words to zero, so a
+// completed call leaves them ready for the next call.
+//
+// A token's K destination rows (and, for E4M3, its scale row) are fetched by
+// the lanes with cp.async into a token ring in shared memory, and that
+// completion is counted on the same mbarrier as the bulk load of the token's
+// first chunk, so everything a stage needs has landed when its phase
+// completes.  The first loads are issued before the per-expert tables are
+// built, which keeps the copy engine busy during the set-up.
+// ---------------------------------------------------------------------------
+// Releases of the token-ordered pipeline happen in batches: once kRelLag +
+// kRelBatch groups are unreleased, one wait, one proxy fence and one gpu-scope
+// fence release every group but the newest kRelLag.
+constexpr int kRelBatch = MOE_PERM_REL_BATCH;
+constexpr int kTokRing = 64;  // tokens whose destination rows are held (until released)
+constexpr int kScRing = kMaxStages;  // tokens whose E4M3 scales are held (until processed)
+constexpr int kRecRing = 64;  // committed bulk groups not yet released
+static_assert(kRecRing > kRelLag + kRelBatch && kTokRing > kMaxStages + kRelLag + kRelBatch,
+              "rings too small for the release lag");
 
-constexpr int kRing = 4;  // tokens whose rows are alive at once: >= kRelLag + 2
+enum : int32_t { kRecNone = 0, kRecToken = 1, kRecPad = 2 };
 
-// Shared-memory tables of one copy pipeline.
 struct PermShared {
   int32_t off[MOE_MAX_EXPERTS + 1];
   int32_t cnt[MOE_MAX_EXPERTS];
   int32_t padpref[MOE_MAX_EXPERTS + 1];
-  int32_t rows[kRing][MOE_MAX_TOPK];
+  int32_t rows[kTokRing][MOE_MAX_TOPK];  // destination rows of token sequence number j % kTokRing
+  int32_t rec[kRecRing][3];              // committed groups: {kind, token seq or first pad, end pad}
+  int32_t stage_grp[kMaxStages];         // group that last read each stage
 };
 
-// One copy pipeline, run by one warp: share c of G of the slots and padding
-// rows.  `smem` is the ring (stages, zero chunk, mbarriers).
-__device__ __forceinline__ void permute_warp(const PermArgs& a, const int64_t c, const int64_t G,
-                                             uint8_t* smem, PermShared& sh) {
-  int32_t* s_off = sh.off;
-  int32_t* s_cnt = sh.cnt;
-  int32_t* s_padpref = sh.padpref;
-  auto& s_rows = sh.rows;
+__device__ __forceinline__ void cp_async4(void* sdst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(sdst)), "l"(gsrc)
+               : "memory");
+}
 
+// The mbarrier's current phase also waits for this thread's earlier cp.async
+// copies (the pending count is raised now and lowered when they land).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Lane 0: waits until every bulk group committed before the newest `newer`
+// ones has finished reading shared memory.
+__device__ __forceinline__ void wait_read_older_than(int newer) {
+  if (newer >= 3) bulk_wait_read<3>();
+  else if (newer == 2) bulk_wait_read<2>();
+  else if (newer == 1) bulk_wait_read<1>();
+  else bulk_wait_read<0>();
+}
+
+__device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, PermShared& sh) {
   const int lane = threadIdx.x & 31;
   const int S = a.stages;
+  const int K = a.K, E = a.E, nch = a.n_chunks;
   uint8_t* stage0 = smem;
   uint8_t* zero = smem + (size_t)S * a.stage_bytes;
   uint64_t* bar = reinterpret_cast<uint64_t*>(zero + a.stage_bytes);
+  float* s_sc = reinterpret_cast<float*>(bar + kMaxStages);  // [kScRing][scale_cols] (E4M3)
 
-  // ---- per-expert tables and the padding prefix sum (one warp) ----
-  const int E = a.E;
-  for (int e = lane; e <= E; e += 32) s_off[e] = __ldg(a.offsets + e);
-  for (int e = lane; e < E; e += 32) s_cnt[e] = __ldg(a.counts + e);
-  __syncwarp();
-  int bad = 0;
-  int run = 0;
-  for (int e0 = 0; e0 < E; e0 += 32) {
-    const int e = e0 + lane;
-    int pad = 0;
-    if (e < E) {
-      pad = (s_off[e + 1] - s_off[e]) - s_cnt[e];
-      if (pad < 0 || pad >= kTile || s_cnt[e] < 0) {
-        bad = 1;
-        pad = 0;
-      }
-    }
-    const int incl = warp_inclusive_scan(pad);
-    if (e < E) s_padpref[e] = run + incl - pad;
-    run += __shfl_sync(0xffffffffu, incl, 31);
-  }
-  if (lane == 0) s_padpref[E] = run;
-  const int64_t P = s_off[E];
-  if (__any_sync(0xffffffffu, bad) || P > a.P_cap || s_off[0] != 0) {
-    if (lane == 0) record_error(a.status, MOE_ERR_BOUNDS);
-    return;
-  }
-  __syncwarp();
+  const int64_t tpt = a.tokens_per_ticket;
+  const int64_t n_tok = (a.T + tpt - 1) / tpt;  // token tickets
+  const int first_batch = a.first_tickets;
 
-  // ---- this CTA's share: an equal run of slots and an equal run of padding rows ----
-  const int64_t TK = a.T * a.K;
-  const int64_t PAD = run;
-  const int64_t s0 = TK * c / G, s1 = TK * (c + 1) / G;      // slots
-  const int64_t q0 = PAD * c / G, q1 = PAD * (c + 1) / G;    // padding indices
-
-  // ---- ring set-up ----
-  for (uint32_t i = lane * 16; i < a.stage_bytes; i += 32 * 16)
-    *reinterpret_cast<uint4*>(zero + i) = make_uint4(0, 0, 0, 0);
-  fence_proxy_async_shared();
+  // ---- barriers and the fixed first batch: the first loads need neither
+  // the tables nor P, nor an atomic ----
+  const int64_t dyn0 = (int64_t)gridDim.x * first_batch;  // first counter-issued ticket
+  uint32_t pend = 0;
   if (lane == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
     fence_mbarrier_init();
+    pend = atomicAdd(a.work, 1u);  // needed only once the batch is used up
   }
   __syncwarp();
+  int64_t k_cur = (int64_t)blockIdx.x * first_batch;  // ticket range in hand
+  int64_t k_end = k_cur + first_batch;
+  int64_t n_tickets = -1;  // known once the tables are built (padding count)
+  int64_t tok_cur = 0, tok_end = 0;  // token range of the ticket in hand
+  bool exhausted = false;
+  bool ok = true;
 
-  const int nch = a.n_chunks;
-  const int64_t t_first = s0 < s1 ? s0 / a.K : 0;
-  const int64_t n_units = s0 < s1 ? ((s1 - 1) / a.K - t_first + 1) * nch : 0;
-  // padding rows issued alongside unit u: [pad_lo(u), pad_lo(u + 1)); all of
-  // them at once when this CTA has no token units
-  auto pad_lo = [&](int64_t u) {
-    return n_units > 0 ? q0 + (q1 - q0) * u / n_units : (u > 0 ? q1 : q0);
+  int64_t n_issued = 0, n_tok_issued = 0;
+  int64_t issue_t = -1;
+  int issue_ch = nch;
+  uint32_t n_commit = 0, n_rel = 0;  // lane 0's bulk-group bookkeeping
+
+  const bool fp8 = a.scale_cols > 0;
+
+  // Warp-uniform.  Next token to load, -1 when the work is exhausted, or -2
+  // when the next ticket is not a token ticket and padding cannot be handled
+  // yet (before the tables exist).
+  auto next_ticket = [&](bool allow_pad, int64_t& k) -> bool {
+    if (k_cur < k_end) {
+      if (!allow_pad && k_cur >= n_tok) return false;
+      k = k_cur++;
+      return true;
+    }
+    if (!allow_pad) return false;  // the pending claim may be a padding ticket
+    k = dyn0 + (int64_t)__shfl_sync(0xffffffffu, pend, 0);
+    if (lane == 0 && k < n_tickets) pend = atomicAdd(a.work, 1u);
+    return true;
   };
 
-  auto unit_token = [&](int64_t u) { return t_first + u / nch; };
-  auto issue_load = [&](int64_t u) {  // lane 0 only
-    const int s = (int)(u % S);
-    const int ch = (int)(u % nch);
-    const uint32_t len = chunk_len(a, ch);
-    const uint8_t* src = a.x + unit_token(u) * a.x_stride_bytes + (int64_t)ch * a.chunk_cap;
-    mbar_arrive_expect_tx(&bar[s], len);
-    bulk_load_g2s(stage0 + (size_t)s * a.stage_bytes, src, len, &bar[s]);
-  };
-
-  // Walks padding indices in increasing order and yields their rows.
+  // ---- padding rows: tables and helpers ----
   struct PadCursor {
     int e;
     __device__ void seek(const int32_t* padpref, int E, int64_t q) {
@@ -198,176 +228,245 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, const int64_t c,
       e = lo;
     }
   };
-  PadCursor issue_cur, rel_cur;
-  issue_cur.seek(s_padpref, E, q0);
-  rel_cur.e = issue_cur.e;
   auto pad_row = [&](PadCursor& cur, int64_t q) -> int64_t {
-    while (q >= s_padpref[cur.e + 1]) ++cur.e;
-    return (int64_t)s_off[cur.e] + s_cnt[cur.e] + (q - s_padpref[cur.e]);
+    while (q >= sh.padpref[cur.e + 1]) ++cur.e;
+    return (int64_t)sh.off[cur.e] + sh.cnt[cur.e] + (q - sh.padpref[cur.e]);
   };
-  // zero rows for padding indices [qa, qb): lanes clear the scale rows, lane 0
-  // bulk-stores the zero chunk over every chunk of each row
-  auto issue_padding = [&](int64_t qa, int64_t qb) {
+  // lane 0: +n for padding indices [qa, qb), one add per run inside one expert
+  auto release_padding = [&](int64_t qa, int64_t qb) {
+    PadCursor cur;
+    cur.seek(sh.padpref, E, qa);
+    int64_t q = qa;
+    while (q < qb) {
+      const int64_t r = pad_row(cur, q);
+      const int64_t q_end = min(qb, (int64_t)sh.padpref[cur.e + 1]);
+      atomic_add_relaxed_gpu(a.tile_ready + r / kTile, (uint32_t)(q_end - q));
+      q = q_end;
+    }
+  };
+  // lane 0: release the groups older than the newest kRelLag once they completed
+  auto retire = [&]() {
+    if (a.tile_ready == nullptr || n_commit - n_rel < (uint32_t)(kRelLag + kRelBatch)) return;
+    bulk_wait_all<kRelLag>();
+    fence_proxy_async_global();
+    fence_acq_rel_gpu();
+    while (n_commit - n_rel > (uint32_t)kRelLag) {
+      const int32_t* rc = sh.rec[n_rel % kRecRing];
+      if (rc[0] == kRecToken) {
+        const int32_t* rows = sh.rows[rc[1] % kTokRing];
+        for (int j = 0; j < K; ++j)
+          if (rows[j] >= 0) atomic_add_relaxed_gpu(a.tile_ready + rows[j] / kTile, 1u);
+      } else if (rc[0] == kRecPad) {
+        release_padding(rc[1], rc[2]);
+      }
+      ++n_rel;
+    }
+  };
+  auto push_rec = [&](int32_t kind, int64_t x0, int64_t x1) {  // lane 0, after a commit
+    int32_t* rc = sh.rec[n_commit % kRecRing];
+    rc[0] = kind;
+    rc[1] = (int32_t)x0;
+    rc[2] = (int32_t)x1;
+    ++n_commit;
+  };
+  // Warp-uniform: zero rows for padding ticket pb, as one bulk group.
+  auto do_padding = [&](int64_t pb) {
+    const int64_t qa = pb * a.pad_per_ticket;
+    const int64_t qb = min(qa + a.pad_per_ticket, (int64_t)sh.padpref[E]);
+    PadCursor cur;
+    cur.seek(sh.padpref, E, qa);
     for (int64_t q = qa; q < qb; ++q) {
-      const int64_t r = pad_row(issue_cur, q);
-      if (a.scale_cols > 0)
+      const int64_t r = pad_row(cur, q);
+      if (fp8)
         for (int cc = lane; cc < a.scale_cols; cc += 32) a.xp_scales[r * a.scale_cols + cc] = 0.0f;
       if (lane == 0)
         for (int ch = 0; ch < nch; ++ch)
           bulk_store_s2g(a.xp + r * a.row_bytes + (int64_t)ch * a.chunk_cap, zero, chunk_len(a, ch));
     }
-  };
-  // +n for padding indices [qa, qb), one add per run inside one expert (all
-  // padding rows of an expert share its last tile)
-  auto release_padding = [&](int64_t qa, int64_t qb) {  // lane 0 only, after the fence
-    int64_t q = qa;
-    while (q < qb) {
-      const int64_t r = pad_row(rel_cur, q);
-      const int64_t q_end = min(qb, (int64_t)s_padpref[rel_cur.e + 1]);
-      atomic_add_relaxed_gpu(a.tile_ready + r / kTile, (uint32_t)(q_end - q));
-      q = q_end;
+    __syncwarp();  // the lanes' scale stores precede lane 0's release
+    if (lane == 0) {
+      bulk_commit();
+      push_rec(kRecPad, qa, qb);
+      retire();
     }
-  };
-  // Release the rows whose bulk-store group belonged to unit ur: the token's
-  // slots (after its last chunk) and the padding rows issued with the unit.
-  auto ring = [&](int64_t t) { return (int)((t - t_first) & (kRing - 1)); };
-  auto release_unit = [&](int64_t ur) {  // lane 0 only
-    fence_acq_rel_gpu();
-    if ((ur % nch) == nch - 1) {
-      const int* rows = s_rows[ring(unit_token(ur))];
-      for (int j = 0; j < a.K; ++j)
-        if (rows[j] >= 0) atomic_add_relaxed_gpu(a.tile_ready + rows[j] / kTile, 1u);
-    }
-    release_padding(pad_lo(ur), pad_lo(ur + 1));
   };
 
-  // Row indices (and FP8 scales) of a token are fetched one token ahead into
-  // registers -- lane j holds slot j -- and published to the shared ring when
-  // the token's first unit starts, so no dependent global load sits between
-  // a landed row and its stores.  Slots outside [s0, s1) read as -1.
-  const bool sc_in_regs = a.scale_cols <= 64;
-  int nxt_r = -1;
-  float nxt_s0 = 0.0f, nxt_s1 = 0.0f, cur_s0 = 0.0f, cur_s1 = 0.0f;
-  auto prefetch = [&](int64_t t) {  // all lanes
-    nxt_r = -1;
-    if (lane < a.K) {
-      const int64_t sl = t * a.K + lane;
-      if (sl >= s0 && sl < s1) nxt_r = (int)checked_row(a, sl);
+  // Warp-uniform: issue the next unit's load (claiming a token when the
+  // current one has no chunk left).  Returns false when nothing was issued.
+  auto issue_next = [&](bool allow_pad) -> bool {
+    if (issue_ch == nch) {
+      int64_t t = -1;
+      while (t < 0) {
+        if (tok_cur < tok_end) {
+          t = tok_cur++;
+          break;
+        }
+        if (exhausted) return false;
+        int64_t k;
+        if (!next_ticket(allow_pad, k)) return false;
+        if (k < n_tok) {
+          tok_cur = k * tpt;
+          tok_end = min(a.T, tok_cur + tpt);
+        } else if (k < n_tickets) {
+          do_padding(k - n_tok);
+        } else {
+          exhausted = true;
+          return false;
+        }
+      }
+      issue_t = t;
+      issue_ch = 0;
     }
-    if (a.scale_cols > 0 && sc_in_regs) {
-      const float* xs = a.x_scales + t * a.xs_stride;
-      nxt_s0 = lane < a.scale_cols ? __ldg(xs + lane) : 0.0f;
-      nxt_s1 = lane + 32 < a.scale_cols ? __ldg(xs + lane + 32) : 0.0f;
+    const int s = (int)(n_issued % S);
+    if (lane == 0 && n_issued >= S)  // the stage's previous group has read it
+      wait_read_older_than((int)(n_commit - 1u - (uint32_t)sh.stage_grp[s]));
+    if (issue_ch == 0) {  // the token's rows (and scales) ride on the same barrier phase
+      const int ring = (int)(n_tok_issued % kTokRing);
+      bool copied = false;
+      if (lane < K) {
+        cp_async4(&sh.rows[ring][lane], a.dst_row + issue_t * K + lane);
+        copied = true;
+      }
+      if (fp8)
+        for (int cc = lane; cc < a.scale_cols; cc += 32) {
+          cp_async4(s_sc + (int)(n_tok_issued % kScRing) * a.scale_cols + cc,
+                    a.x_scales + issue_t * a.xs_stride + cc);
+          copied = true;
+        }
+      if (copied) cp_async_arrive(&bar[s]);
+      ++n_tok_issued;
+      __syncwarp();
     }
+    if (lane == 0) {
+      const uint32_t len = chunk_len(a, issue_ch);
+      mbar_arrive_expect_tx(&bar[s], len);
+      bulk_load_g2s(stage0 + (size_t)s * a.stage_bytes,
+                    a.x + issue_t * a.x_stride_bytes + (int64_t)issue_ch * a.chunk_cap, len,
+                    &bar[s]);
+    }
+    ++issue_ch;
+    ++n_issued;
+    return true;
   };
-  auto publish = [&](int64_t t) {  // all lanes
-    if (lane < a.K) s_rows[ring(t)][lane] = nxt_r;
-    cur_s0 = nxt_s0;
-    cur_s1 = nxt_s1;
-    __syncwarp();
-  };
-  const int64_t t_last = n_units > 0 ? unit_token(n_units - 1) : -1;
-  if (n_units > 0) {
-    prefetch(t_first);
-    publish(t_first);
-    if (t_first + 1 <= t_last) prefetch(t_first + 1);
+
+  // ---- first loads, from the first claimed batch (token tickets only) ----
+  while (n_issued < S && issue_next(false)) {
   }
 
-  int64_t issued = 0;
-  if (lane == 0)
-    for (; issued < n_units && issued < S; ++issued) issue_load(issued);
-
-  int64_t u_fail = -1;
-  for (int64_t u = 0; u < n_units; ++u) {
-    const int s = (int)(u % S);
-    const uint32_t parity = (uint32_t)((u / S) & 1);
-    if (u > 0 && (u % nch) == 0) {  // first unit of a new token
-      const int64_t tn = unit_token(u);
-      publish(tn);
-      if (tn + 1 <= t_last) prefetch(tn + 1);
+  // ---- per-expert tables, the padding prefix sum and the zero chunk ----
+  for (int e = lane; e <= E; e += 32) sh.off[e] = __ldg(a.offsets + e);
+  for (int e = lane; e < E; e += 32) sh.cnt[e] = __ldg(a.counts + e);
+  __syncwarp();
+  int bad = 0;
+  int run = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    int pad = 0;
+    if (e < E) {
+      pad = (sh.off[e + 1] - sh.off[e]) - sh.cnt[e];
+      if (pad < 0 || pad >= kTile || sh.cnt[e] < 0) {
+        bad = 1;
+        pad = 0;
+      }
     }
-    // padding first: it needs no load, so it keeps the copy engine busy
-    issue_padding(pad_lo(u), pad_lo(u + 1));
-    int ok = 1;
-    if (lane == 0) ok = mbar_wait_bounded(&bar[s], parity) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) {
-      u_fail = u;
+    const int incl = warp_inclusive_scan(pad);
+    if (e < E) sh.padpref[e] = run + incl - pad;
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) sh.padpref[E] = run;
+  for (uint32_t i = lane * 16; i < a.stage_bytes; i += 32 * 16)
+    *reinterpret_cast<uint4*>(zero + i) = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_shared();
+  __syncwarp();
+  if (__any_sync(0xffffffffu, bad) || (int64_t)sh.off[E] > a.P_cap || sh.off[0] != 0) {
+    if (lane == 0) record_error(a.status, MOE_ERR_BOUNDS);
+    ok = false;  // nothing is stored; the loads already issued drain below
+  }
+  n_tickets = n_tok + ((int64_t)run + a.pad_per_ticket - 1) / a.pad_per_ticket;
+
+  // ---- main loop: process unit u, then top the ring up ----
+  int64_t u = 0;
+  while (ok) {
+    if (u == n_issued && !issue_next(true)) break;
+    const int s = (int)(u % S);
+    int landed = 1;
+    if (lane == 0) landed = mbar_wait_bounded(&bar[s], (uint32_t)((u / S) & 1)) ? 1 : 0;
+    landed = __shfl_sync(0xffffffffu, landed, 0);
+    if (!landed) {
+      if (lane == 0) record_error(a.status, MOE_ERR_TIMEOUT);
+      ok = false;
       break;
     }
-    const int64_t t = unit_token(u);
+    mbar_try_wait(&bar[s], (uint32_t)((u / S) & 1));  // every lane acquires the landed phase
+    const int64_t j = u / nch;
     const int ch = (int)(u % nch);
-    const int* rows = s_rows[ring(t)];
-
-    if (ch == 0 && a.scale_cols > 0) {  // FP8 scale row, all lanes
-      for (int j = 0; j < a.K; ++j) {
-        const int64_t r = rows[j];
-        if (r < 0) continue;
-        float* dst = a.xp_scales + r * a.scale_cols;
-        if (sc_in_regs) {
-          if (lane < a.scale_cols) dst[lane] = cur_s0;
-          if (lane + 32 < a.scale_cols) dst[lane + 32] = cur_s1;
-        } else {
-          for (int cc = lane; cc < a.scale_cols; cc += 32)
-            dst[cc] = __ldg(a.x_scales + t * a.xs_stride + cc);
+    int32_t* rows = sh.rows[j % kTokRing];
+    if (ch == 0) {  // checked once per token: an out-of-range row is reported and skipped
+      if (lane < K) {
+        const int32_t r = rows[lane];
+        if (r != -1 && (r < 0 || (int64_t)r >= a.P_cap)) {
+          record_error(a.status, MOE_ERR_BOUNDS);
+          rows[lane] = -1;
         }
+      }
+      __syncwarp();
+      if (fp8) {
+        const float* sc = s_sc + (j % kScRing) * a.scale_cols;
+        for (int k = 0; k < K; ++k) {
+          const int64_t r = rows[k];
+          if (r < 0) continue;
+          for (int cc = lane; cc < a.scale_cols; cc += 32) a.xp_scales[r * a.scale_cols + cc] = sc[cc];
+        }
+        __syncwarp();  // the lanes' scale stores precede lane 0's release
       }
     }
     if (lane == 0) {
       const uint32_t len = chunk_len(a, ch);
       const uint8_t* src = stage0 + (size_t)s * a.stage_bytes;
-      for (int j = 0; j < a.K; ++j) {
-        const int64_t r = rows[j];
+      for (int k = 0; k < K; ++k) {
+        const int64_t r = rows[k];
         if (r < 0) continue;
         bulk_store_s2g(a.xp + r * a.row_bytes + (int64_t)ch * a.chunk_cap, src, len);
       }
       bulk_commit();
+      sh.stage_grp[s] = (int32_t)n_commit;
+      push_rec(ch == nch - 1 ? kRecToken : kRecNone, j, 0);
+      retire();
     }
-    if (a.tile_ready) {
-      __syncwarp();  // the lanes' scale stores precede lane 0's release
-      if (lane == 0) {
-        bulk_wait_all<kRelLag>();  // groups <= u - kRelLag have completed
-        fence_proxy_async_global();
-        if (u >= kRelLag) release_unit(u - kRelLag);
-      }
-    }
-    if (lane == 0) {
-      bulk_wait_read<kReadLag>();  // the stores of unit u-kReadLag have read their stage
-      if (u >= kReadLag && issued < n_units) {
-        issue_load(issued);  // lands in the stage unit u-kReadLag used
-        ++issued;
-      }
+    ++u;
+    while (n_issued < u + S && issue_next(true)) {
     }
   }
 
-  if (u_fail >= 0) {
-    if (lane == 0) {
-      record_error(a.status, MOE_ERR_TIMEOUT);
-      bulk_wait_all<0>();
-      // give the other loads still in flight a bounded chance to land before
-      // the CTA's shared memory is released
-      for (int64_t u = u_fail + 1; u < issued; ++u)
-        if (!mbar_wait_bounded(&bar[u % S], (uint32_t)((u / S) & 1))) break;
-    }
-    return;
-  }
-  if (n_units == 0) {  // no token rows here: all of this CTA's padding at once
-    issue_padding(q0, q1);
-    if (lane == 0) bulk_commit();
-  }
-
-  // ---- drain, then release what is still pending ----
+  // ---- drain ----
   __syncwarp();
   if (lane == 0) {
+    if (!ok) {
+      // loads still in flight get a bounded chance to land before the CTA's
+      // shared memory is given back
+      for (int64_t v = u; v < n_issued; ++v)
+        if (!mbar_wait_bounded(&bar[v % S], (uint32_t)((v / S) & 1))) break;
+    }
     bulk_wait_all<0>();
-    if (a.tile_ready) {
+    if (ok && a.tile_ready != nullptr && n_commit != n_rel) {
       fence_proxy_async_global();
-      if (n_units > 0) {
-        for (int64_t ur = max((int64_t)0, n_units - kRelLag); ur < n_units; ++ur) release_unit(ur);
-      } else {
-        fence_acq_rel_gpu();
-        release_padding(q0, q1);
+      fence_acq_rel_gpu();
+      while (n_rel != n_commit) {
+        const int32_t* rc = sh.rec[n_rel % kRecRing];
+        if (rc[0] == kRecToken) {
+          const int32_t* rws = sh.rows[rc[1] % kTokRing];
+          for (int k = 0; k < K; ++k)
+            if (rws[k] >= 0) atomic_add_relaxed_gpu(a.tile_ready + rws[k] / kTile, 1u);
+        } else if (rc[0] == kRecPad) {
+          release_padding(rc[1], rc[2]);
+        }
+        ++n_rel;
       }
+    }
+    // the last CTA out returns the claim counter and the done count to zero
+    if (atomic_add_acq_rel_gpu(a.work + 1, 1u) == gridDim.x - 1) {
+      a.work[0] = 0u;
+      a.work[1] = 0u;
     }
   }
 }
@@ -376,7 +475,7 @@ __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
   pdl_begin();
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ PermShared sh;
-  permute_warp(a, blockIdx.x, gridDim.x, smem, sh);
+  permute_warp(a, smem, sh);
 }
 
 // ---------------------------------------------------------------------------
@@ -689,6 +788,7 @@ int make_perm_args(const void* x, int dtype, int64_t T, int H, int64_t x_row_str
                    int K, const int32_t* expert_counts, const int32_t* expert_offsets, int E,
                    void* xp, float* xp_scales, int64_t P_cap, uint32_t* tile_ready,
                    int32_t* d_status, PermArgs* out) {
+  *out = PermArgs{};
   if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_E4M3) return MOE_ERR_UNSUPPORTED;
   if (T < 0 || H <= 0 || K < 1 || K > MOE_MAX_TOPK || E < 1 || E > MOE_MAX_EXPERTS)
     return MOE_ERR_INVALID_ARG;
@@ -736,15 +836,18 @@ int make_perm_args(const void* x, int dtype, int64_t T, int H, int64_t x_row_str
   return MOE_OK;
 }
 
-// Ring depth for `ctas_per_sm` CTAs sharing an SM's shared memory; returns the
-// dynamic shared-memory bytes, or 0 if even two stages do not fit.
-size_t size_ring(PermArgs& a, int ctas_per_sm, size_t static_smem, int optin) {
+// Ring depth for `ctas_per_sm` CTAs sharing an SM's shared memory, with
+// `extra` bytes of dynamic shared memory after the stages, the zero chunk and
+// the kMaxStages mbarriers; returns the dynamic shared-memory bytes, or 0 if
+// even two stages do not fit.
+size_t size_ring(PermArgs& a, int ctas_per_sm, size_t static_smem, int optin, size_t extra = 0) {
+  const size_t fixed = (size_t)a.stage_bytes + kMaxStages * 8 + extra;
   const size_t per_cta = (size_t)optin / ctas_per_sm - static_smem - 1024;
-  int stages = (int)((per_cta - a.stage_bytes - kMaxStages * 8) / a.stage_bytes);
+  int stages = per_cta > fixed ? (int)((per_cta - fixed) / a.stage_bytes) : 0;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) stages = 2;
   a.stages = stages;
-  const size_t dyn = (size_t)(stages + 1) * a.stage_bytes + (size_t)stages * 8;
+  const size_t dyn = (size_t)stages * a.stage_bytes + fixed;
   return dyn + static_smem > (size_t)optin ? 0 : dyn;
 }
 
@@ -785,22 +888,35 @@ extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
                                     int64_t x_scales_row_stride, const int32_t* dst_row, int K,
                                     const int32_t* expert_counts, const int32_t* expert_offsets,
                                     int E, void* xp, float* xp_scales, int64_t P_cap,
-                                    uint32_t* tile_ready, int32_t* d_status, void* stream) {
+                                    uint32_t* tile_ready, uint32_t* work, int32_t* d_status,
+                                    void* stream) {
   using namespace moe;
   PermArgs a;
   int st = make_perm_args(x, dtype, T, H, x_row_stride, x_scales, x_scales_row_stride, dst_row,
                           K, expert_counts, expert_offsets, E, xp, xp_scales, P_cap, tile_ready,
                           d_status, &a);
   if (st != MOE_OK) return st;
+  if (!work || !moe_host::aligned4(work)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;  // P = 0: nothing to write
 
   const int dev = moe_host::current_device();
   const int optin = optin_smem(dev);
   if (optin < 0) return MOE_ERR_CUDA;
   const int ctas_per_sm = perm_ctas_per_sm(a.row_bytes);
-  const size_t dyn = size_ring(a, ctas_per_sm, sizeof(PermShared), optin);
+  const size_t scale_ring = (size_t)kScRing * a.scale_cols * sizeof(float);
+  const size_t dyn = size_ring(a, ctas_per_sm, sizeof(PermShared), optin, scale_ring);
   if (dyn == 0) return MOE_ERR_UNSUPPORTED;
   if (!allow_max_dyn_smem(permute_kernel, dev, optin, g_dyn_perm)) return MOE_ERR_CUDA;
+
+  // Tickets: a token ticket names enough tokens for about 32 KiB of row
+  // writes; a padding ticket names as many rows as a token ticket writes.
+  const int64_t tok_bytes = (int64_t)K * a.row_bytes;
+  a.tokens_per_ticket = std::min<int64_t>(64, std::max<int64_t>(1, (32768 + tok_bytes - 1) / tok_bytes));
+  a.pad_per_ticket = (int64_t)K * a.tokens_per_ticket;
+  a.first_tickets = (int)std::max<int64_t>(
+      1, (a.stages + (int64_t)a.n_chunks * a.tokens_per_ticket - 1) /
+             ((int64_t)a.n_chunks * a.tokens_per_ticket));
+  a.work = work;
 
   const int64_t v_bound = T * K + (int64_t)(kTile - 1) * E;
   int64_t grid = (int64_t)moe_host::sm_count(dev) * ctas_per_sm;

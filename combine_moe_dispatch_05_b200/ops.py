@@ -35,7 +35,7 @@ SIGNATURES = {
     "moe_dispatch_layout_static": (_int, [_vp, _i64, _int, _int, _int, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp, _i64, _vp, _vp]),
     "moe_dispatch_permute": (_int, [_vp, _int, _i64, _int, _i64, _vp, _i64, _vp, _int, _vp, _vp,
-                                    _int, _vp, _vp, _i64, _vp, _vp, _vp]),
+                                    _int, _vp, _vp, _i64, _vp, _vp, _vp, _vp]),
     "moe_dispatch_permute_consume": (_int, [_vp, _int, _i64, _int, _i64, _vp, _i64, _vp, _int,
                                             _vp, _vp, _int, _vp, _vp, _vp, _i64, _vp, _vp, _i64,
                                             _vp, _vp]),
@@ -158,6 +158,7 @@ class Layout:
     row_src: Optional[torch.Tensor]
     tile_ready: Optional[torch.Tensor]
     workspace: Optional[torch.Tensor]   # None for layouts filled by moe_dispatch_layout_static
+    work: torch.Tensor                  # permute's scheduling words: int32 [2], zero between calls
 
 
 def alloc_layout(T: int, K: int, E: int, R: int, device, P_cap: Optional[int] = None,
@@ -173,7 +174,7 @@ def alloc_layout(T: int, K: int, E: int, R: int, device, P_cap: Optional[int] = 
         torch.empty(max(P_cap, 1), **i32) if with_row_src else None,
         torch.empty(max((P_cap + TILE - 1) // TILE, 1), dtype=torch.int32, device=device)
         if with_counters else None,
-        ws)
+        ws, torch.zeros(2, **i32))
 
 
 def moe_dispatch_layout(topk_idx: torch.Tensor, E: int, R: int, layout: Optional[Layout] = None,
@@ -247,7 +248,8 @@ def moe_dispatch_permute(x: torch.Tensor, L: Layout, xp: Optional[torch.Tensor] 
     rc = lib().moe_dispatch_permute(
         _ptr(x), dt, T, H, x.stride(0), _ptr(x_scales), xs_stride, _ptr(L.dst_row), L.K,
         _ptr(L.expert_counts), _ptr(L.expert_offsets), L.E, _ptr(xp), _ptr(xp_scales), L.P_cap,
-        _ptr(L.tile_ready) if use_counters else None, _ptr(status), _stream(stream))
+        _ptr(L.tile_ready) if use_counters else None, _ptr(L.work), _ptr(status),
+        _stream(stream))
     _check(rc, "moe_dispatch_permute")
     return (xp, xp_scales) if dt == DTYPE_E4M3 else xp
 

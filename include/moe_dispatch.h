@@ -203,8 +203,17 @@ MOE_API int moe_dispatch_layout_static(const int32_t* topk_idx, int64_t T, int K
  *   tile_ready (nullable) counters zeroed by the layout call; each finished
  *            row adds 1 to tile_ready[row/128] after its bytes (and scales)
  *            are globally visible, behind a gpu-scope release (a
- *            fence.acq_rel.gpu per token, then relaxed atomic adds), so a
- *            tile whose counter reads 128 with an ld.acquire.gpu is complete.
+ *            fence.acq_rel.gpu per group of rows, then relaxed atomic adds),
+ *            so a tile whose counter reads 128 with an ld.acquire.gpu is
+ *            complete.
+ * Scheduling words:
+ *   work     device uint32 [2], 4-byte aligned, non-NULL: the claim counter
+ *            through which the copy pipelines take tokens and padding rows as
+ *            they go (so pipelines on faster SMs take more of the work), and
+ *            a count of finished pipelines.  They must be zero before the
+ *            first call that uses them; every completed call returns them to
+ *            zero.  Calls that share the same words must not overlap on the
+ *            GPU (order them on one stream, or give each its own words).
  * Data errors: MOE_ERR_BOUNDS if a dst_row entry or offset leaves
  *   [0, P_cap) (that write is skipped); MOE_ERR_TIMEOUT if a staged load
  *   did not land within about 2 s (outputs and device state are then
@@ -214,8 +223,8 @@ MOE_API int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H, int
                          const float* x_scales, int64_t x_scales_row_stride,
                          const int32_t* dst_row, int K, const int32_t* expert_counts,
                          const int32_t* expert_offsets, int E, void* xp, float* xp_scales,
-                         int64_t P_cap, uint32_t* tile_ready, int32_t* d_status,
-                         void* stream);
+                         int64_t P_cap, uint32_t* tile_ready, uint32_t* work,
+                         int32_t* d_status, void* stream);
 
 /*
  * Counter-driven overlap: the dispatch permute and a consumer of its

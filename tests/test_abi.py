@@ -71,13 +71,16 @@ def test_host_argument_errors_launch_nothing():
                          null) == ops.ERR_INVALID_ARG
     # bad dtype
     assert L.moe_dispatch_permute(fake, 7, 4, 64, 64, null, 0, fake, 2, fake, fake, 4, fake,
-                                  null, 1024, null, null, null) == ops.ERR_UNSUPPORTED
+                                  null, 1024, null, fake, null, null) == ops.ERR_UNSUPPORTED
     # E4M3 needs H % 128 == 0
     assert L.moe_dispatch_permute(fake, 1, 4, 64, 64, fake, 0, fake, 2, fake, fake, 4, fake,
-                                  fake, 1024, null, null, null) == ops.ERR_INVALID_ARG
+                                  fake, 1024, null, fake, null, null) == ops.ERR_INVALID_ARG
     # row stride smaller than H
     assert L.moe_dispatch_permute(fake, 0, 4, 64, 32, null, 0, fake, 2, fake, fake, 4, fake,
-                                  null, 1024, null, null, null) == ops.ERR_INVALID_ARG
+                                  null, 1024, null, fake, null, null) == ops.ERR_INVALID_ARG
+    # no scheduling words
+    assert L.moe_dispatch_permute(fake, 0, 4, 64, 64, null, 0, fake, 2, fake, fake, 4, fake,
+                                  null, 1024, null, null, null, null) == ops.ERR_INVALID_ARG
     assert L.moe_quantize_e4m3(fake, 4, 100, 100, fake, fake, null, null) == ops.ERR_INVALID_ARG
     assert L.moe_combine_bwd(fake, fake, fake, fake, fake, fake, 4, 4, 2, 64, 128, fake, fake,
                              null, null) == ops.ERR_CAPACITY
