@@ -51,21 +51,47 @@ struct QuantPermArgs {
   int chunk;          // channels per unit: H, or kQpChunk when H is larger
   int stage_bytes;    // chunk codes + chunk/128 scales, rounded up to 16
   int bulk_scales;    // scales go out by bulk store (H % 512 == 0, aligned base)
+  uint32_t* work;     // [2] claim counter and done count
+  int64_t tokens_per_ticket;
+  int64_t pad_per_ticket;
 };
 
 __host__ __device__ constexpr int qp_stage_bytes(int chunk) {
   return (chunk + chunk / 32 + 15) / 16 * 16;
 }
 
-__global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPermArgs a) {
+// Work claiming and releases (as in the token-ordered permute): CTA c starts
+// with token ticket c, every later ticket comes from the claim counter
+// work[0] (ticket G + the counter's old value); tickets [0, n_tok) name tpt
+// tokens each, tickets [n_tok, n_tok + n_pad) name ppt padding rows each.
+// Thread 0 resolves the token after next while the CTA works on the current
+// one, so the claim's latency is hidden.  Rows are released in batches: once
+// kQRelLag + kQRelBatch bulk groups are unreleased, one completion wait and
+// one gpu-scope fence release all but the newest kQRelLag.  The last CTA out
+// returns work[0..1] to zero.
+constexpr int kQRing = 16;       // tokens whose rows are held (until released)
+constexpr int kQRelLag = 4;      // bulk groups left in flight at a release
+constexpr int kQRelBatch = 8;    // groups released per completion wait
+static_assert(kQRing > kQRelLag + kQRelBatch + 2, "token ring too small for the release lag");
+
+__device__ __forceinline__ uint32_t qp_atom_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+__global__ void __launch_bounds__(kQpThreads, 8) permute_quant_kernel(const QuantPermArgs a) {
   pdl_begin();
   extern __shared__ __align__(128) uint8_t qp_stage[];
-  __shared__ int32_t s_row[4][MOE_MAX_TOPK];
+  __shared__ int32_t s_row[kQRing][MOE_MAX_TOPK];
+  __shared__ int64_t s_tok[kQRing];   // token of local sequence number j % kQRing, -1 = none
   __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_cnt[MOE_MAX_EXPERTS];
   __shared__ int32_t s_pad[MOE_MAX_EXPERTS];
   __shared__ int32_t s_padpref[MOE_MAX_EXPERTS + 1];
   __shared__ int32_t s_warp[kQpThreads / 32];
+  __shared__ int64_t s_padq;          // padding ticket being processed, -1 = none
+  __shared__ int32_t s_rec[kQRelLag + kQRelBatch];  // per unreleased group: its token's slot or -1
   __shared__ int s_bad;
 
   const int tid = threadIdx.x, lane = tid & 31;
@@ -74,8 +100,15 @@ __global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPe
   const int CH = a.chunk;
   const int nch = (H + CH - 1) / CH;
   const unsigned half_mask = 0xFFFFu << (lane & 16);
+  const int64_t tpt = a.tokens_per_ticket, ppt = a.pad_per_ticket;
+  const int64_t n_tok = (a.T + tpt - 1) / tpt;
+  const int64_t dyn0 = gridDim.x;  // first counter-issued ticket
 
-  if (tid == 0) s_bad = 0;
+  uint32_t pend = 0;  // thread 0: the claim in flight
+  if (tid == 0) {
+    s_bad = 0;
+    pend = atomicAdd(a.work, 1u);
+  }
   for (int e = tid; e <= E; e += kQpThreads) s_off[e] = __ldg(a.offsets + e);
   for (int e = tid; e < E; e += kQpThreads) s_cnt[e] = __ldg(a.counts + e);
   __syncthreads();
@@ -87,18 +120,44 @@ __global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPe
   }
   __syncthreads();
   block_exclusive_scan(s_pad, E, s_padpref, s_warp);
-  if (s_bad || (int64_t)s_off[E] > a.P_cap || s_off[0] != 0) {
-    if (tid == 0) record_error(a.status, MOE_ERR_BOUNDS);
-    return;
-  }
+  const bool bad = s_bad || (int64_t)s_off[E] > a.P_cap || s_off[0] != 0;
+  if (bad && tid == 0) record_error(a.status, MOE_ERR_BOUNDS);
+  const int pad_total = s_padpref[E];
+  const int64_t n_tickets = n_tok + ((int64_t)pad_total + ppt - 1) / ppt;
 
-  // Row indices of a token sit in a ring of four: the slot of local token j
-  // is filled at the start of token j-1 and rewritten at the start of token
-  // j+3.  Thread 0 reads it to issue token j's stores (after each of token
-  // j's barriers) and to release its rows (after the first barrier of token
-  // j+1), both before it reaches the last barrier of token j+2.
+  // ---- thread 0's ticket stream ----
+  int64_t k_cur = blockIdx.x, k_end = blockIdx.x + 1;  // fixed first ticket
+  int64_t tok_cur = 0, tok_end = 0;
+  int64_t first_pad_ticket = -1;  // the ticket that ended the token phase
+  bool tokens_done = false;
+  auto take_ticket = [&]() -> int64_t {  // thread 0
+    if (k_cur < k_end) return k_cur++;
+    const int64_t k = dyn0 + (int64_t)pend;
+    if (k < n_tickets) pend = atomicAdd(a.work, 1u);
+    return k;
+  };
+  auto next_token = [&]() -> int64_t {  // thread 0; -1 when the token tickets are used up
+    while (!tokens_done) {
+      if (tok_cur < tok_end) return tok_cur++;
+      const int64_t k = take_ticket();
+      if (k < n_tok) {
+        tok_cur = k * tpt;
+        tok_end = min(a.T, tok_cur + tpt);
+      } else {
+        tokens_done = true;
+        first_pad_ticket = k;
+      }
+    }
+    return -1;
+  };
+  if (tid == 0) {
+    s_tok[0] = bad ? -1 : next_token();
+    s_tok[1] = (bad || s_tok[0] < 0) ? -1 : next_token();
+  }
+  __syncthreads();
+
   auto fetch = [&](int64_t t, int slot) {
-    if (tid < K && t < a.T) {
+    if (tid < K && t >= 0) {
       int r = __ldg(a.dst_row + t * K + tid);
       if (r != -1 && (r < 0 || (int64_t)r >= a.P_cap)) {
         record_error(a.status, MOE_ERR_BOUNDS);
@@ -107,19 +166,35 @@ __global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPe
       s_row[slot][tid] = r;
     }
   };
-  auto release_rows = [&](const int32_t* rows) {  // thread 0, after its group completed
+  // thread 0: group bookkeeping for batched releases
+  uint32_t n_commit = 0, n_rel = 0;
+  auto release_batch = [&](uint32_t keep) {  // thread 0: release all groups but the newest `keep`
+    if (keep == 0) bulk_wait_all<0>(); else bulk_wait_all<kQRelLag>();
     fence_proxy_async_global();
     fence_acq_rel_gpu();
-    for (int k = 0; k < K; ++k)
-      if (rows[k] >= 0) atomic_add_relaxed_gpu(a.tile_ready + rows[k] / kTile, 1u);
+    while (n_commit - n_rel > keep) {
+      const int32_t slot = s_rec[n_rel % (kQRelLag + kQRelBatch)];
+      if (slot >= 0)
+        for (int k = 0; k < K; ++k) {
+          const int32_t r = s_row[slot][k];
+          if (r >= 0) atomic_add_relaxed_gpu(a.tile_ready + r / kTile, 1u);
+        }
+      ++n_rel;
+    }
   };
 
-  fetch(blockIdx.x, 0);
+  fetch(s_tok[0], 0);
   __syncthreads();
-  int slot = 0;
   int64_t u = 0;  // units issued by this CTA
-  for (int64_t t = blockIdx.x; t < a.T; t += gridDim.x) {
-    fetch(t + gridDim.x, (slot + 1) & 3);
+  for (int64_t j = 0;; ++j) {
+    const int64_t t = s_tok[j % kQRing];
+    if (t < 0) break;
+    const int slot = (int)(j % kQRing);
+    fetch(s_tok[(j + 1) % kQRing], (int)((j + 1) % kQRing));
+    if (tid == 0) {  // the token after next
+      const int64_t t1 = s_tok[(j + 1) % kQRing];
+      s_tok[(j + 2) % kQRing] = t1 < 0 ? -1 : next_token();
+    }
     const int32_t* rows = s_row[slot];
     const uint16_t* xr = a.x + t * a.x_stride;
     for (int c = 0; c < nch; ++c, ++u) {
@@ -185,22 +260,19 @@ __global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPe
             bulk_store_s2g(a.xp_scales + r * nb + (c0 >> 7), st_scl, (uint32_t)(cl >> 5));
         }
         bulk_commit();
-        if (a.tile_ready && c == 0 && u > 0) {
-          // the previous unit was the last of this CTA's previous token
-          bulk_wait_all<1>();
-          release_rows(s_row[(slot + 3) & 3]);
-        }
+        s_rec[n_commit % (kQRelLag + kQRelBatch)] = c == nch - 1 ? slot : -1;
+        ++n_commit;
+        if (a.tile_ready && n_commit - n_rel == (uint32_t)(kQRelLag + kQRelBatch))
+          release_batch(kQRelLag);
       }
     }
-    slot = (slot + 1) & 3;
   }
   if (tid == 0) {
-    bulk_wait_all<0>();  // stages stay alive until read; the last token's rows are written
-    if (a.tile_ready && u > 0) release_rows(s_row[(slot + 3) & 3]);
+    if (a.tile_ready) release_batch(0);  // the last tokens' rows: written, then released
+    else bulk_wait_all<0>();             // stages stay alive until read; rows written
   }
 
-  // ---- padding rows: code 0x00, scale 0 ----
-  const int pad_total = s_padpref[E];
+  // ---- padding rows: code 0x00, scale 0, claimed ppt rows at a time ----
   const int Vc = H >> 4;  // 16-byte code vectors per row
   auto pad_row = [&](int q) -> int64_t {
     int lo = 0, hi = E - 1;  // last expert with padpref <= q
@@ -210,18 +282,44 @@ __global__ void __launch_bounds__(kQpThreads) permute_quant_kernel(const QuantPe
     }
     return (int64_t)s_off[lo] + s_cnt[lo] + (q - s_padpref[lo]);
   };
-  for (int q = blockIdx.x; q < pad_total; q += gridDim.x) {
-    const int64_t r = pad_row(q);
-    for (int v = tid; v < Vc; v += kQpThreads) st_v4(a.xp + r * H + (int64_t)v * 16, make_uint4(0, 0, 0, 0));
-    for (int b = tid; b < nb; b += kQpThreads) a.xp_scales[r * nb + b] = 0.0f;
-  }
-  if (a.tile_ready && (int)blockIdx.x < pad_total) {
-    __syncthreads();  // all of this CTA's padding rows are written
-    if (tid == 0) {
-      fence_acq_rel_gpu();
-      for (int q = blockIdx.x; q < pad_total; q += gridDim.x)
-        atomic_add_relaxed_gpu(a.tile_ready + pad_row(q) / kTile, 1u);
+  if (tid == 0) s_padq = (!bad && first_pad_ticket >= n_tok && first_pad_ticket < n_tickets)
+                             ? first_pad_ticket - n_tok : -1;
+  __syncthreads();
+  while (true) {
+    const int64_t pq = s_padq;
+    if (pq < 0) break;
+    const int q0 = (int)(pq * ppt), q1 = (int)min((int64_t)pad_total, (pq + 1) * ppt);
+    for (int q = q0; q < q1; ++q) {
+      const int64_t r = pad_row(q);
+      for (int v = tid; v < Vc; v += kQpThreads) st_v4(a.xp + r * H + (int64_t)v * 16, make_uint4(0, 0, 0, 0));
+      for (int b = tid; b < nb; b += kQpThreads) a.xp_scales[r * nb + b] = 0.0f;
     }
+    __syncthreads();  // every row of the ticket is written (and s_padq read by all)
+    if (tid == 0) {
+      if (a.tile_ready) {
+        fence_acq_rel_gpu();
+        for (int q = q0; q < q1;) {  // one add per run inside one expert
+          const int64_t r = pad_row(q);
+          int lo = 0, hi = E - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_padpref[mid] <= q) lo = mid; else hi = mid - 1;
+          }
+          const int qe = min(q1, s_padpref[lo + 1]);
+          atomic_add_relaxed_gpu(a.tile_ready + r / kTile, (uint32_t)(qe - q));
+          q = qe;
+        }
+      }
+      const int64_t k = take_ticket();
+      s_padq = (k >= n_tok && k < n_tickets) ? k - n_tok : -1;
+    }
+    __syncthreads();
+  }
+
+  // the last CTA out returns the claim counter and the done count to zero
+  if (tid == 0 && qp_atom_add_acq_rel(a.work + 1, 1u) == gridDim.x - 1) {
+    a.work[0] = 0u;
+    a.work[1] = 0u;
   }
 }
 
@@ -235,7 +333,7 @@ extern "C" int moe_dispatch_permute_quant(const void* x, int64_t T, int H, int64
                                           const int32_t* expert_counts,
                                           const int32_t* expert_offsets, int E, void* xp,
                                           float* xp_scales, int64_t P_cap, uint32_t* tile_ready,
-                                          int32_t* d_status, void* stream) {
+                                          uint32_t* work, int32_t* d_status, void* stream) {
   using namespace moe;
   if (T < 0 || H <= 0 || H % 128 != 0 || K < 1 || K > MOE_MAX_TOPK || E < 1 ||
       E > MOE_MAX_EXPERTS || x_row_stride < H || x_row_stride % 8 != 0)
@@ -248,6 +346,7 @@ extern "C" int moe_dispatch_permute_quant(const void* x, int64_t T, int H, int64
     return MOE_ERR_INVALID_ARG;
   if (!moe_host::aligned16(xp) || (x && !moe_host::aligned16(x)) || !moe_host::aligned4(xp_scales))
     return MOE_ERR_INVALID_ARG;
+  if (!work || !moe_host::aligned4(work)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   QuantPermArgs a;
   a.x = static_cast<const uint16_t*>(x);
@@ -267,6 +366,12 @@ extern "C" int moe_dispatch_permute_quant(const void* x, int64_t T, int H, int64
   a.chunk = H < kQpChunk ? H : kQpChunk;
   a.stage_bytes = qp_stage_bytes(a.chunk);
   a.bulk_scales = (H % 512 == 0 && moe_host::aligned16(xp_scales)) ? 1 : 0;
+  a.work = work;
+  // a token ticket names about 32 KiB of code writes; a padding ticket 32 rows
+  const int64_t tok_bytes = (int64_t)K * H;
+  a.tokens_per_ticket = (32768 + tok_bytes - 1) / tok_bytes;
+  if (a.tokens_per_ticket > 64) a.tokens_per_ticket = 64;
+  a.pad_per_ticket = 32;
   const size_t dyn = (size_t)kQpStages * a.stage_bytes;
   // occupancy at the largest stage size, so one cached figure holds for every H
   const size_t dyn_max = (size_t)kQpStages * qp_stage_bytes(kQpChunk);

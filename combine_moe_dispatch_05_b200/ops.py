@@ -40,7 +40,7 @@ SIGNATURES = {
                                             _vp, _vp, _int, _vp, _vp, _vp, _i64, _vp, _vp, _i64,
                                             _vp, _vp]),
     "moe_dispatch_permute_quant": (_int, [_vp, _i64, _int, _i64, _vp, _int, _vp, _vp, _int, _vp,
-                                          _vp, _i64, _vp, _vp, _vp]),
+                                          _vp, _i64, _vp, _vp, _vp, _vp]),
     "moe_combine": (_int, [_vp, _vp, _vp, _vp, _i64, _int, _int, _i64, _vp, _vp, _vp]),
     "moe_combine_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _i64, _int, _int, _i64, _vp,
                                _vp, _vp, _vp]),
@@ -318,7 +318,8 @@ def moe_dispatch_permute_quant(x: torch.Tensor, L: Layout, xp: Optional[torch.Te
     rc = lib().moe_dispatch_permute_quant(
         _ptr(x), T, H, x.stride(0), _ptr(L.dst_row), L.K, _ptr(L.expert_counts),
         _ptr(L.expert_offsets), L.E, _ptr(xp), _ptr(xp_scales), L.P_cap,
-        _ptr(L.tile_ready) if use_counters else None, _ptr(status), _stream(stream))
+        _ptr(L.tile_ready) if use_counters else None, _ptr(L.work), _ptr(status),
+        _stream(stream))
     _check(rc, "moe_dispatch_permute_quant")
     return xp, xp_scales
 

@@ -274,7 +274,8 @@ MOE_API int moe_dispatch_permute_consume(const void* x, int dtype, int64_t T, in
  *      16-byte aligned; H % 128 == 0.
  * Out: xp uint8 [P_cap, H] (16-byte aligned); xp_scales fp32 [P_cap, H/128]
  *      (4-byte aligned; with 16-byte alignment and H % 512 == 0 the scales
- *      are bulk-stored with the codes); tile_ready (nullable) as in
+ *      are bulk-stored with the codes); tile_ready (nullable) and work
+ *      (scheduling words, uint32 [2], zero between calls) as in
  *      moe_dispatch_permute.
  * Data errors: MOE_ERR_BOUNDS as in moe_dispatch_permute.
  */
@@ -283,7 +284,7 @@ MOE_API int moe_dispatch_permute_quant(const void* x, int64_t T, int H, int64_t 
                                        const int32_t* expert_counts,
                                        const int32_t* expert_offsets, int E, void* xp,
                                        float* xp_scales, int64_t P_cap, uint32_t* tile_ready,
-                                       int32_t* d_status, void* stream);
+                                       uint32_t* work, int32_t* d_status, void* stream);
 
 /*
  * Combine ([ASC] function description, expert_scales, shared_expert_x):
