@@ -15,9 +15,9 @@ permute -> combine: dispatch + combine, the metric's pair) the same way over
 the same number of steps.  Inputs are resident in HBM when the timed region
 starts; L2 is flushed (256 MiB write) before every timed step and the flush
 is outside the timed events.  Inside the timed region the only events are
-one before and one after each step; per-kernel times (phases_us, and the
-roofline's dominant kernel) come from a separate pass right after it with an
-event between every two kernels.  With N GPUs (torchrun), every rank runs its
+one before and one after each step; per-kernel times (phases_us: medians;
+the roofline's dominant kernel: its mean) come from a separate pass right
+after it with an event between every two kernels.  With N GPUs (torchrun), every rank runs its
 own replica on its own data (weak scaling; no collective on the data path);
 the reported time is the max over ranks.
 
@@ -323,11 +323,16 @@ def run_ours(args, world, rank, local):
         ops.moe_dispatch_permute(x, L, xp=xp, status=st)
         ops.moe_combine(xp, L.dst_row, sc, out=out, status=st)
 
+    def dispatch():  # layout -> permute, chained
+        ops.moe_dispatch_layout(ids, E, R, layout=L, status=st)
+        ops.moe_dispatch_permute(x, L, xp=xp, status=st)
+
     with ClockSampler(smi_id(torch, dev)) as clk:
         step_ms = timed_steps(graph.replay if graph is not None else step)
         # The forward step alone (layout -> permute -> combine), timed the same
         # way over the same number of steps; with --fwd-only it is the step.
         fwd_ms = step_ms if args.fwd_only else timed_steps(forward)
+        disp_ms = timed_steps(dispatch)
     if ops.read_status(st) != 0:
         raise RuntimeError(f"device status {ops.read_status(st)} in the timed steps")
     snapshot = None
@@ -365,9 +370,14 @@ def run_ours(args, world, rank, local):
     value = bytes_step * world / (ms_per_step * 1e-3) / 1e9
     tok_s = T * world / (ms_per_step * 1e-3)
 
-    phase_us = {p: 1e3 * statistics.mean(v) for p, v in per_phase.items()}
+    # per-kernel medians (a rare launch in this pass takes several times its
+    # usual time, which would move a mean); the roofline uses the mean launch
+    # duration of its kernel
+    phase_us = {p: 1e3 * statistics.median(v) for p, v in per_phase.items()}
+    phase_mean_us = {p: 1e3 * statistics.mean(v) for p, v in per_phase.items()}
     phase_gbs = {p: nbytes[p] / (phase_us[p] * 1e-6) / 1e9 for p in phases}
     dom = max((p for p in phases if p != "layout"), key=lambda p: phase_us[p])
+    dom_gbs = nbytes[dom] / (phase_mean_us[dom] * 1e-6) / 1e9
     peak, peak_src = measured_peak()
     fwd_bytes = sum(nbytes[p] for p in ("layout", "permute", "combine"))
     fwd_ms_per_step = max_over_ranks(sum(fwd_ms), world) / args.steps
@@ -380,8 +390,14 @@ def run_ours(args, world, rank, local):
                 "what": "layout -> permute -> combine chained on one stream, no events between "
                         "the kernels, L2 flushed before each step (outside the events); max "
                         "over ranks"}
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(phase_gbs[dom], 1),
-                "peak": peak, "unit": "GB/s", "frac": round(phase_gbs[dom] / peak, 4),
+    disp_bytes = nbytes["layout"] + nbytes["permute"]
+    disp_ms_per_step = max_over_ranks(sum(disp_ms), world) / args.steps
+    disp_gbs = disp_bytes * world / (disp_ms_per_step * 1e-3) / 1e9
+    dispatch_step = {"ms": round(disp_ms_per_step, 5), "GBps": round(disp_gbs, 1),
+                     "frac": round(disp_gbs / world / peak, 4), "bytes": disp_bytes,
+                     "what": "layout -> permute chained, timed like fwd_step"}
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src ==
                 "measured" else "fallback 6.65 TB/s",
                 "traffic": ncu_traffic(dom),
@@ -405,15 +421,18 @@ def run_ours(args, world, rank, local):
                                 "eager launches (programmatic dependent launch)",
                       "parallelism": f"replicas x{world}"},
            "phases_us": {p: round(v, 2) for p, v in phase_us.items()},
-           "phases_note": f"per-kernel pass of {n_phase} steps with an event between every two "
-                          f"kernels (which serialises them): {phase_step_ms:.4f} ms per step "
-                          "there, against ms_per_step in the timed region",
+           "phases_us_mean_max": {p: [round(phase_mean_us[p], 2), round(1e3 * max(v), 2)]
+                                  for p, v in per_phase.items()},
+           "phases_note": f"medians of a per-kernel pass of {n_phase} steps with an event between "
+                          f"every two kernels (which serialises them): {phase_step_ms:.4f} ms "
+                          "per step there, against ms_per_step in the timed region",
            "phases_gbs": {p: round(v, 1) for p, v in phase_gbs.items()},
            "groups_gbs": groups_gbs(nbytes, phase_us),
            "roofline": roofline,
            "fwd_step": fwd_step,
+           "dispatch_step": dispatch_step,
            "gpu_launches": LAUNCHES_PER_STEP[args.fwd_only] * args.steps +
-           (0 if args.fwd_only else LAUNCHES_PER_STEP[True] * args.steps),
+           (0 if args.fwd_only else LAUNCHES_PER_STEP[True] * args.steps) + 3 * args.steps,
            "clocks": clk.summary()}
     if snapshot is not None:
         res["_timed_outputs"] = snapshot

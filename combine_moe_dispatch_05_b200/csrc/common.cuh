@@ -72,6 +72,53 @@ __device__ __forceinline__ void atomic_add_relaxed_gpu(uint32_t* p, uint32_t v) 
   asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
+// ------------------------------------------------------- work claiming --
+// The kernels that split their work dynamically share one protocol over two
+// caller-provided words: work[0] is a claim counter, work[1] counts CTAs
+// that are done.  Both are zero when a launch starts.  CTA c first takes the
+// fixed tickets [c*b, c*b + b) (no atomic, so its first loads go out at
+// once); every later ticket is dyn0 + the old value of work[0] (dyn0 = G*b),
+// claimed one ticket ahead so the atomic's latency is hidden.  Tickets past
+// the work are discarded.  The last CTA to finish returns both words to
+// zero: its acq_rel add on work[1] comes after every other CTA's, and each
+// of those follows all of that CTA's claims.
+struct TicketStream {  // one thread's view (the CTA's issuing thread)
+  uint32_t* work;
+  int64_t k_cur, k_end, dyn0;
+  uint32_t pend;
+
+  __device__ void init(uint32_t* w, int64_t first_batch) {
+    work = w;
+    k_cur = (int64_t)blockIdx.x * first_batch;
+    k_end = k_cur + first_batch;
+    dyn0 = (int64_t)gridDim.x * first_batch;
+    pend = atomicAdd(w, 1u);
+  }
+  // Next ticket; a new claim is issued only while tickets below `limit`
+  // may still exist.
+  __device__ int64_t take(int64_t limit) {
+    if (k_cur < k_end) return k_cur++;
+    const int64_t k = dyn0 + (int64_t)pend;
+    if (k < limit) pend = atomicAdd(work, 1u);
+    return k;
+  }
+};
+
+// Called once per CTA by its issuing thread after its last claim.
+__device__ __forceinline__ void finish_claims(uint32_t* work) {
+  if (atomic_add_acq_rel_gpu(work + 1, 1u) == gridDim.x - 1) {
+    work[0] = 0u;
+    work[1] = 0u;
+  }
+}
+
 // ----------------------------------------------------------- shared mem --
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

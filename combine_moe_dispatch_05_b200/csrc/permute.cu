@@ -149,12 +149,6 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
 // Lane 0: waits until every bulk group committed before the newest `newer`
 // ones has finished reading shared memory.
 __device__ __forceinline__ void wait_read_older_than(int newer) {
@@ -463,11 +457,7 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
         ++n_rel;
       }
     }
-    // the last CTA out returns the claim counter and the done count to zero
-    if (atomic_add_acq_rel_gpu(a.work + 1, 1u) == gridDim.x - 1) {
-      a.work[0] = 0u;
-      a.work[1] = 0u;
-    }
+    finish_claims(a.work);  // the last CTA out returns both words to zero
   }
 }
 

@@ -60,10 +60,9 @@ __host__ __device__ constexpr int qp_stage_bytes(int chunk) {
   return (chunk + chunk / 32 + 15) / 16 * 16;
 }
 
-// Work claiming and releases (as in the token-ordered permute): CTA c starts
-// with token ticket c, every later ticket comes from the claim counter
-// work[0] (ticket G + the counter's old value); tickets [0, n_tok) name tpt
-// tokens each, tickets [n_tok, n_tok + n_pad) name ppt padding rows each.
+// Work claiming (TicketStream, first batch of one ticket) and releases, as in
+// the token-ordered permute: tickets [0, n_tok) name tpt tokens each, tickets
+// [n_tok, n_tok + n_pad) name ppt padding rows each.
 // Thread 0 resolves the token after next while the CTA works on the current
 // one, so the claim's latency is hidden.  Rows are released in batches: once
 // kQRelLag + kQRelBatch bulk groups are unreleased, one completion wait and
@@ -73,12 +72,6 @@ constexpr int kQRing = 16;       // tokens whose rows are held (until released)
 constexpr int kQRelLag = 4;      // bulk groups left in flight at a release
 constexpr int kQRelBatch = 8;    // groups released per completion wait
 static_assert(kQRing > kQRelLag + kQRelBatch + 2, "token ring too small for the release lag");
-
-__device__ __forceinline__ uint32_t qp_atom_add_acq_rel(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
 
 __global__ void __launch_bounds__(kQpThreads, 8) permute_quant_kernel(const QuantPermArgs a) {
   pdl_begin();
@@ -102,12 +95,11 @@ __global__ void __launch_bounds__(kQpThreads, 8) permute_quant_kernel(const Quan
   const unsigned half_mask = 0xFFFFu << (lane & 16);
   const int64_t tpt = a.tokens_per_ticket, ppt = a.pad_per_ticket;
   const int64_t n_tok = (a.T + tpt - 1) / tpt;
-  const int64_t dyn0 = gridDim.x;  // first counter-issued ticket
 
-  uint32_t pend = 0;  // thread 0: the claim in flight
+  __shared__ TicketStream tk;  // used by thread 0 only
   if (tid == 0) {
     s_bad = 0;
-    pend = atomicAdd(a.work, 1u);
+    tk.init(a.work, 1);
   }
   for (int e = tid; e <= E; e += kQpThreads) s_off[e] = __ldg(a.offsets + e);
   for (int e = tid; e < E; e += kQpThreads) s_cnt[e] = __ldg(a.counts + e);
@@ -126,16 +118,10 @@ __global__ void __launch_bounds__(kQpThreads, 8) permute_quant_kernel(const Quan
   const int64_t n_tickets = n_tok + ((int64_t)pad_total + ppt - 1) / ppt;
 
   // ---- thread 0's ticket stream ----
-  int64_t k_cur = blockIdx.x, k_end = blockIdx.x + 1;  // fixed first ticket
   int64_t tok_cur = 0, tok_end = 0;
   int64_t first_pad_ticket = -1;  // the ticket that ended the token phase
   bool tokens_done = false;
-  auto take_ticket = [&]() -> int64_t {  // thread 0
-    if (k_cur < k_end) return k_cur++;
-    const int64_t k = dyn0 + (int64_t)pend;
-    if (k < n_tickets) pend = atomicAdd(a.work, 1u);
-    return k;
-  };
+  auto take_ticket = [&]() -> int64_t { return tk.take(n_tickets); };  // thread 0
   auto next_token = [&]() -> int64_t {  // thread 0; -1 when the token tickets are used up
     while (!tokens_done) {
       if (tok_cur < tok_end) return tok_cur++;
@@ -316,11 +302,7 @@ __global__ void __launch_bounds__(kQpThreads, 8) permute_quant_kernel(const Quan
     __syncthreads();
   }
 
-  // the last CTA out returns the claim counter and the done count to zero
-  if (tid == 0 && qp_atom_add_acq_rel(a.work + 1, 1u) == gridDim.x - 1) {
-    a.work[0] = 0u;
-    a.work[1] = 0u;
-  }
+  if (tid == 0) finish_claims(a.work);  // the last CTA out returns both words to zero
 }
 
 std::atomic<int> g_occ_qp[moe_host::kMaxCachedDevices];

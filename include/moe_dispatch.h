@@ -306,7 +306,8 @@ MOE_API int moe_combine(const void* y, const int32_t* dst_row, const float* scal
 
 /*
  * Backward of combine (out is linear in y and in scales):
- *   grad_y[dst_row[t*K+k]] = bf16( scales[t,k] * grad_out[t] )   (fp32 product)
+ *   grad_y[dst_row[t*K+k]] = bf16( scales[t,k] * grad_out[t] )   (the exact
+ *                            product, rounded once to nearest-even)
  *   grad_scales[t*K+k]     = sum_h grad_out[t,h] * y[dst_row[t*K+k], h]
  *                            (fp32, fixed order for a given H)
  *   padding rows of grad_y below P are set to 0; rows >= P untouched.
