@@ -64,4 +64,5 @@ def test_step_in_cuda_graph_matches_eager():
             assert torch.equal(a, b)
         results.append(P)
     assert ops.read_status(st) == 0
+    assert int(L.work.abs().sum().item()) == 0  # the permute's words are back to zero
     del graph
