@@ -12,21 +12,24 @@
 //     drives the SM's bulk-copy (TMA) unit: a non-multicast cp.async.bulk
 //     global -> shared load of each token row (or 16 KiB column chunk) into
 //     an S-stage ring, completed on an mbarrier, then K cp.async.bulk
-//     shared -> global stores of the same bytes, one per destination row.  The row is read from HBM once and
-//     never passes through registers.
+//     shared -> global stores of the same bytes, one per destination row.
+//     The row is read from HBM once and never passes through registers; the
+//     token's destination rows (and E4M3 scales) arrive by cp.async on the
+//     same mbarrier phase.
 //   * padding rows are bulk-stored from a zero-filled shared chunk.
-//   * every CTA takes an equal contiguous run of the T*K slots and an equal
-//     run of the padding rows, so each writes the same number of rows of
-//     each kind whatever the expert skew; a CTA's padding rows are issued a
-//     few at a time ahead of each token unit's load wait, which keeps the
-//     copy engine busy while the load is in flight.
+//   * work is claimed dynamically: tokens, then padding rows, as tickets
+//     from a claim counter, so CTAs on faster SMs take more of it and all
+//     finish together (see the token-ordered pipeline below).
 //   * counters: a row's +1 is released only after its bulk-store group has
-//     completed (cp.async.bulk.wait_group), behind a proxy fence, with a lag
-//     of a few groups so the copy pipeline never drains.  The release is one
-//     fence.acq_rel.gpu per token followed by relaxed adds (the pull
-//     request's atom.acq_rel.gpu on every add is a full fence per row).  FP8
-//     scale rows are copied by the 32 lanes with plain stores before the
-//     same release.
+//     completed (cp.async.bulk.wait_group), behind a proxy fence; releases
+//     are batched (one completion wait and one fence.acq_rel.gpu per 8
+//     groups, 4 groups behind) followed by relaxed adds (the pull request's
+//     atom.acq_rel.gpu on every add is a full fence per row).  FP8 scale
+//     rows are copied by the 32 lanes with plain stores before the same
+//     release.
+//   * the tile-ordered pipeline for the counter-driven overlap (at the end of
+//     this file) fills 16-row items in tile order and releases each as it
+//     lands.
 #include <algorithm>
 
 #include "common.cuh"
