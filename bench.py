@@ -6,9 +6,9 @@
 A step is one pass of the whole path over one batch of the DeepSeek-V3-shaped
 decode workload (T=4096 tokens, H=7168, E=256 experts, K=8, 8 logical EP
 ranks, Zipf(0.6) routing):
-    layout -> permute (bf16, with chunk-completion counters) -> combine
-    (identity experts: y = the dispatched rows) -> combine backward ->
-    dispatch backward.
+    layout -> permute (bf16, with chunk-completion counters; one
+    moe_dispatch call) -> combine (identity experts: y = the dispatched
+    rows) -> combine backward -> dispatch backward.
 value = algorithmic HBM bytes of the step / device time of the step, in GB/s
 (also reported: tokens/s).  fwd_step times the forward pair alone (layout ->
 permute -> combine: dispatch + combine, the metric's pair) the same way over
@@ -264,11 +264,17 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream()
 
     def step(evs=None):
+        # the timed steps use the one-call dispatch (layout + permute, the
+        # permute's first loads overlapping the layout); the per-kernel pass
+        # calls the two separately to put an event between them
         rec = (lambda i: evs[i].record(stream)) if evs else (lambda i: None)
         rec(0)
-        ops.moe_dispatch_layout(ids, E, R, layout=L, status=st)
-        rec(1)
-        ops.moe_dispatch_permute(x, L, xp=xp, status=st)
+        if evs:
+            ops.moe_dispatch_layout(ids, E, R, layout=L, status=st)
+            rec(1)
+            ops.moe_dispatch_permute(x, L, xp=xp, status=st)
+        else:
+            ops.moe_dispatch(ids, x, E, R, layout=L, xp=xp, status=st)
         rec(2)
         ops.moe_combine(xp, L.dst_row, sc, out=out, status=st)   # identity experts: y = xp
         rec(3)
@@ -319,13 +325,11 @@ def run_ours(args, world, rank, local):
         return [a.elapsed_time(b) for a, b in bounds]
 
     def forward():  # dispatch + combine: the metric's pair, chained
-        ops.moe_dispatch_layout(ids, E, R, layout=L, status=st)
-        ops.moe_dispatch_permute(x, L, xp=xp, status=st)
+        ops.moe_dispatch(ids, x, E, R, layout=L, xp=xp, status=st)
         ops.moe_combine(xp, L.dst_row, sc, out=out, status=st)
 
-    def dispatch():  # layout -> permute, chained
-        ops.moe_dispatch_layout(ids, E, R, layout=L, status=st)
-        ops.moe_dispatch_permute(x, L, xp=xp, status=st)
+    def dispatch():  # layout -> permute in one call
+        ops.moe_dispatch(ids, x, E, R, layout=L, xp=xp, status=st)
 
     with ClockSampler(smi_id(torch, dev)) as clk:
         step_ms = timed_steps(graph.replay if graph is not None else step)
@@ -387,15 +391,15 @@ def run_ours(args, world, rank, local):
                 "tokens_per_s": round(T * world / (fwd_ms_per_step * 1e-3), 1),
                 "bytes": fwd_bytes, "steps": args.steps,
                 "median_ms": round(statistics.median(fwd_ms), 5),
-                "what": "layout -> permute -> combine chained on one stream, no events between "
-                        "the kernels, L2 flushed before each step (outside the events); max "
-                        "over ranks"}
+                "what": "layout -> permute (one moe_dispatch call) -> combine chained on one "
+                        "stream, no events between the kernels, L2 flushed before each step "
+                        "(outside the events); max over ranks"}
     disp_bytes = nbytes["layout"] + nbytes["permute"]
     disp_ms_per_step = max_over_ranks(sum(disp_ms), world) / args.steps
     disp_gbs = disp_bytes * world / (disp_ms_per_step * 1e-3) / 1e9
     dispatch_step = {"ms": round(disp_ms_per_step, 5), "GBps": round(disp_gbs, 1),
                      "frac": round(disp_gbs / world / peak, 4), "bytes": disp_bytes,
-                     "what": "layout -> permute chained, timed like fwd_step"}
+                     "what": "layout -> permute in one moe_dispatch call, timed like fwd_step"}
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1),
                 "peak": peak, "unit": "GB/s", "frac": round(dom_gbs / peak, 4),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src ==

@@ -35,6 +35,13 @@ __device__ __forceinline__ void pdl_begin() {
 }
 
 
+// Lets the next kernel in the stream launch now (its CTAs park in their own
+// pdl_begin until this grid has finished).  Used only by the layout kernels
+// inside the combined dispatch call, right after their pdl_begin.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- status --
 __device__ __forceinline__ void record_error(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(reinterpret_cast<int*>(status), 0, code);
@@ -306,6 +313,24 @@ namespace moe_host {
 int sm_count(int device);
 int current_device();
 int launch_status();  // MOE_OK or MOE_ERR_CUDA from cudaGetLastError()
+
+}  // namespace moe_host
+
+// Host launchers shared by the separate calls and the combined dispatch call.
+namespace moe {
+int layout_launch(const int32_t* topk_idx, int64_t T, int K, int E, int R,
+                  int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                  int32_t* rank_offsets, int32_t* dst_row, int32_t* row_src,
+                  uint32_t* tile_ready, int64_t P_cap, int32_t* d_status, void* workspace,
+                  size_t workspace_bytes, cudaStream_t s, int trigger, int dry_run);
+int permute_launch(const void* x, int dtype, int64_t T, int H, int64_t x_row_stride,
+                   const float* x_scales, int64_t x_scales_row_stride, const int32_t* dst_row,
+                   int K, const int32_t* expert_counts, const int32_t* expert_offsets, int E,
+                   void* xp, float* xp_scales, int64_t P_cap, uint32_t* tile_ready,
+                   uint32_t* work, int32_t* d_status, cudaStream_t s, int early_x, int dry_run);
+}  // namespace moe
+
+namespace moe_host {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

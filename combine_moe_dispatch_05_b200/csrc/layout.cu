@@ -116,8 +116,9 @@ layout_count_kernel(const int32_t* __restrict__ ids, int64_t T, int K, int E,
                     int tokens_per_block, int32_t* __restrict__ block_counts,
                     int32_t* __restrict__ slot_rank, int32_t* __restrict__ row_src,
                     int64_t P_cap, uint32_t* __restrict__ tile_ready, int64_t n_tiles,
-                    int32_t* status) {
+                    int32_t* status, int trigger) {
   pdl_begin();
+  if (trigger) pdl_trigger();
   __shared__ __align__(16) uint16_t hist[kLayoutWarps * MOE_MAX_EXPERTS];  // [warp][E]
   __shared__ int32_t s_ids[kSlotsPerBlock];
 
@@ -186,8 +187,10 @@ layout_assign_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict_
                      int R, int tokens_per_block, int32_t* __restrict__ expert_counts,
                      int32_t* __restrict__ expert_offsets, int32_t* __restrict__ rank_counts,
                      int32_t* __restrict__ rank_offsets, int32_t* __restrict__ dst_row,
-                     int32_t* __restrict__ row_src, int64_t P_cap, int32_t* status) {
+                     int32_t* __restrict__ row_src, int64_t P_cap, int32_t* status,
+                     int trigger) {
   pdl_begin();
+  if (trigger) pdl_trigger();
   __shared__ int32_t s_pre[kLayoutThreads];   // [group][E] partial sums of earlier blocks
   __shared__ int32_t s_tot[kLayoutThreads];   // [group][E] partial sums of all blocks
   __shared__ int32_t s_base[MOE_MAX_EXPERTS];
@@ -312,13 +315,15 @@ extern "C" size_t moe_layout_workspace_bytes(int64_t T, int K, int E) {
          moe::align256((size_t)(T > 0 ? T : 1) * K * sizeof(int32_t));
 }
 
-extern "C" int moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int K, int E, int R,
-                                   int32_t* expert_counts, int32_t* expert_offsets,
-                                   int32_t* rank_counts, int32_t* rank_offsets,
-                                   int32_t* dst_row, int32_t* row_src, uint32_t* tile_ready,
-                                   int64_t P_cap, int32_t* d_status, void* workspace,
-                                   size_t workspace_bytes, void* stream) {
-  using namespace moe;
+namespace moe {
+// The layout's checks and launches (see moe_dispatch_layout).  With dry_run
+// the checks run and nothing is launched; with trigger both kernels let the
+// next kernel in the stream launch right after their own grid wait.
+int layout_launch(const int32_t* topk_idx, int64_t T, int K, int E, int R,
+                  int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                  int32_t* rank_offsets, int32_t* dst_row, int32_t* row_src,
+                  uint32_t* tile_ready, int64_t P_cap, int32_t* d_status, void* workspace,
+                  size_t workspace_bytes, cudaStream_t s, int trigger, int dry_run) {
   if (T < 0 || K < 1 || K > MOE_MAX_TOPK || E < 1 || E > MOE_MAX_EXPERTS || R < 1 || R > E ||
       E % R != 0)
     return MOE_ERR_INVALID_ARG;
@@ -336,8 +341,8 @@ extern "C" int moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int K, in
                         (const void*)tile_ready})
     if (!moe_host::aligned4(q)) return MOE_ERR_INVALID_ARG;
   if (workspace_bytes < moe_layout_workspace_bytes(T, K, E)) return MOE_ERR_INVALID_ARG;
+  if (dry_run) return MOE_OK;
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t n_tiles = (P_cap + kTile - 1) / kTile;
   const int tpb = tokens_per_block_for(K);
   const int nb = T > 0 ? (int)((T + tpb - 1) / tpb) : 1;
@@ -347,12 +352,24 @@ extern "C" int moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int K, in
 
   int st = moe_host::launch(layout_count_kernel, dim3(nb), dim3(kLayoutThreads), 0, s, topk_idx, T,
                             K, E, tpb, block_counts, slot_rank, row_src, P_cap, tile_ready,
-                            n_tiles, d_status);
+                            n_tiles, d_status, trigger);
   if (st != MOE_OK) return st;
   return moe_host::launch(layout_assign_kernel, dim3(nb), dim3(kLayoutThreads), 0, s, topk_idx,
                           (const int32_t*)slot_rank, (const int32_t*)block_counts, nb, T, K, E, R,
                           tpb, expert_counts, expert_offsets, rank_counts, rank_offsets, dst_row,
-                          row_src, P_cap, d_status);
+                          row_src, P_cap, d_status, trigger);
+}
+}  // namespace moe
+
+extern "C" int moe_dispatch_layout(const int32_t* topk_idx, int64_t T, int K, int E, int R,
+                                   int32_t* expert_counts, int32_t* expert_offsets,
+                                   int32_t* rank_counts, int32_t* rank_offsets,
+                                   int32_t* dst_row, int32_t* row_src, uint32_t* tile_ready,
+                                   int64_t P_cap, int32_t* d_status, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return moe::layout_launch(topk_idx, T, K, E, R, expert_counts, expert_offsets, rank_counts,
+                            rank_offsets, dst_row, row_src, tile_ready, P_cap, d_status,
+                            workspace, workspace_bytes, static_cast<cudaStream_t>(stream), 0, 0);
 }
 
 // ---------------------------------------------------------------------------

@@ -90,6 +90,7 @@ struct PermArgs {
   int64_t tokens_per_ticket; // tokens named by one token ticket
   int64_t pad_per_ticket;    // padding rows named by one padding ticket
   int first_tickets;         // tickets each CTA claims at once to fill its ring
+  int early_x;               // issue the first batch's x loads before the grid wait
 };
 
 __device__ __forceinline__ uint32_t chunk_len(const PermArgs& a, int ch) {
@@ -139,6 +140,7 @@ struct PermShared {
   int32_t rows[kTokRing][MOE_MAX_TOPK];  // destination rows of token sequence number j % kTokRing
   int32_t rec[kRecRing][3];              // committed groups: {kind, token seq or first pad, end pad}
   int32_t stage_grp[kMaxStages];         // group that last read each stage
+  int32_t pre_tok[kMaxStages];           // tokens loaded before the grid wait (early_x)
 };
 
 __device__ __forceinline__ void cp_async4(void* sdst, const void* gsrc) {
@@ -181,7 +183,6 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
   if (lane == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
     fence_mbarrier_init();
-    pend = atomicAdd(a.work, 1u);  // needed only once the batch is used up
   }
   __syncwarp();
   int64_t k_cur = (int64_t)blockIdx.x * first_batch;  // ticket range in hand
@@ -290,7 +291,7 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
 
   // Warp-uniform: issue the next unit's load (claiming a token when the
   // current one has no chunk left).  Returns false when nothing was issued.
-  auto issue_next = [&](bool allow_pad) -> bool {
+  auto issue_next = [&](bool allow_pad, bool with_rows) -> bool {
     if (issue_ch == nch) {
       int64_t t = -1;
       while (t < 0) {
@@ -317,7 +318,10 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
     const int s = (int)(n_issued % S);
     if (lane == 0 && n_issued >= S)  // the stage's previous group has read it
       wait_read_older_than((int)(n_commit - 1u - (uint32_t)sh.stage_grp[s]));
-    if (issue_ch == 0) {  // the token's rows (and scales) ride on the same barrier phase
+    if (issue_ch == 0 && !with_rows) {  // rows and scales are read after the grid wait
+      if (lane == 0) sh.pre_tok[n_tok_issued] = (int32_t)issue_t;
+      ++n_tok_issued;
+    } else if (issue_ch == 0) {  // the token's rows (and scales) ride on the same barrier phase
       const int ring = (int)(n_tok_issued % kTokRing);
       bool copied = false;
       if (lane < K) {
@@ -347,8 +351,27 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
   };
 
   // ---- first loads, from the first claimed batch (token tickets only) ----
-  while (n_issued < S && issue_next(false)) {
+  // With early_x (only inside the combined dispatch call, where x was written
+  // before the layout's kernels started) these loads go out before the grid
+  // wait, while the layout still runs; the tokens' rows and scales, which
+  // the layout produces or which are only needed later, are then read right
+  // after the wait.  Otherwise the grid wait came first.
+  const bool pre = a.early_x != 0;
+  while (n_issued < S && issue_next(false, !pre)) {
   }
+  if (pre) {
+    pdl_begin();
+    __syncwarp();
+    for (int64_t j = 0; j < n_tok_issued; ++j) {
+      const int64_t t = sh.pre_tok[j];
+      if (lane < K) sh.rows[j % kTokRing][lane] = __ldg(a.dst_row + t * K + lane);
+      if (fp8)
+        for (int cc = lane; cc < a.scale_cols; cc += 32)
+          s_sc[(j % kScRing) * a.scale_cols + cc] = __ldg(a.x_scales + t * a.xs_stride + cc);
+    }
+    __syncwarp();
+  }
+  if (lane == 0) pend = atomicAdd(a.work, 1u);  // needed only once the batch is used up
 
   // ---- per-expert tables, the padding prefix sum and the zero chunk ----
   for (int e = lane; e <= E; e += 32) sh.off[e] = __ldg(a.offsets + e);
@@ -384,7 +407,7 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
   // ---- main loop: process unit u, then top the ring up ----
   int64_t u = 0;
   while (ok) {
-    if (u == n_issued && !issue_next(true)) break;
+    if (u == n_issued && !issue_next(true, true)) break;
     const int s = (int)(u % S);
     int landed = 1;
     if (lane == 0) landed = mbar_wait_bounded(&bar[s], (uint32_t)((u / S) & 1)) ? 1 : 0;
@@ -431,7 +454,7 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
       retire();
     }
     ++u;
-    while (n_issued < u + S && issue_next(true)) {
+    while (n_issued < u + S && issue_next(true, true)) {
     }
   }
 
@@ -465,7 +488,7 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
 }
 
 __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
-  pdl_begin();
+  if (!a.early_x) pdl_begin();  // with early_x, permute_warp waits after its first loads
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ PermShared sh;
   permute_warp(a, smem, sh);
@@ -876,21 +899,25 @@ std::atomic<int> g_dyn_consume[moe_host::kMaxCachedDevices];
 }  // namespace
 }  // namespace moe
 
-extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
-                                    int64_t x_row_stride, const float* x_scales,
-                                    int64_t x_scales_row_stride, const int32_t* dst_row, int K,
-                                    const int32_t* expert_counts, const int32_t* expert_offsets,
-                                    int E, void* xp, float* xp_scales, int64_t P_cap,
-                                    uint32_t* tile_ready, uint32_t* work, int32_t* d_status,
-                                    void* stream) {
-  using namespace moe;
+namespace moe {
+// The permute's checks and launch (see moe_dispatch_permute).  With dry_run
+// the checks run and nothing is launched; early_x lets the kernel issue its
+// first x loads before its grid wait, which only a caller that launched the
+// layout itself may ask for (x must be complete before the previous kernel
+// began).
+int permute_launch(const void* x, int dtype, int64_t T, int H, int64_t x_row_stride,
+                   const float* x_scales, int64_t x_scales_row_stride, const int32_t* dst_row,
+                   int K, const int32_t* expert_counts, const int32_t* expert_offsets, int E,
+                   void* xp, float* xp_scales, int64_t P_cap, uint32_t* tile_ready,
+                   uint32_t* work, int32_t* d_status, cudaStream_t stream, int early_x,
+                   int dry_run) {
   PermArgs a;
   int st = make_perm_args(x, dtype, T, H, x_row_stride, x_scales, x_scales_row_stride, dst_row,
                           K, expert_counts, expert_offsets, E, xp, xp_scales, P_cap, tile_ready,
                           d_status, &a);
   if (st != MOE_OK) return st;
   if (!work || !moe_host::aligned4(work)) return MOE_ERR_INVALID_ARG;
-  if (T == 0) return MOE_OK;  // P = 0: nothing to write
+  if (dry_run || T == 0) return MOE_OK;  // T = 0: P = 0, nothing to write
 
   const int dev = moe_host::current_device();
   const int optin = optin_smem(dev);
@@ -910,14 +937,27 @@ extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
       1, (a.stages + (int64_t)a.n_chunks * a.tokens_per_ticket - 1) /
              ((int64_t)a.n_chunks * a.tokens_per_ticket));
   a.work = work;
+  a.early_x = early_x;
 
   const int64_t v_bound = T * K + (int64_t)(kTile - 1) * E;
   int64_t grid = (int64_t)moe_host::sm_count(dev) * ctas_per_sm;
   const int64_t by_work = (v_bound + 7) / 8;
   if (grid > by_work) grid = by_work;
   if (grid < 1) grid = 1;
-  return moe_host::launch(permute_kernel, dim3((unsigned)grid), dim3(32), dyn,
-                          static_cast<cudaStream_t>(stream), a);
+  return moe_host::launch(permute_kernel, dim3((unsigned)grid), dim3(32), dyn, stream, a);
+}
+}  // namespace moe
+
+extern "C" int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H,
+                                    int64_t x_row_stride, const float* x_scales,
+                                    int64_t x_scales_row_stride, const int32_t* dst_row, int K,
+                                    const int32_t* expert_counts, const int32_t* expert_offsets,
+                                    int E, void* xp, float* xp_scales, int64_t P_cap,
+                                    uint32_t* tile_ready, uint32_t* work, int32_t* d_status,
+                                    void* stream) {
+  return moe::permute_launch(x, dtype, T, H, x_row_stride, x_scales, x_scales_row_stride,
+                             dst_row, K, expert_counts, expert_offsets, E, xp, xp_scales, P_cap,
+                             tile_ready, work, d_status, static_cast<cudaStream_t>(stream), 0, 0);
 }
 
 extern "C" int moe_dispatch_permute_consume(

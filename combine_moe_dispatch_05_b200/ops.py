@@ -36,6 +36,9 @@ SIGNATURES = {
                                           _vp, _vp, _i64, _vp, _vp]),
     "moe_dispatch_permute": (_int, [_vp, _int, _i64, _int, _i64, _vp, _i64, _vp, _int, _vp, _vp,
                                     _int, _vp, _vp, _i64, _vp, _vp, _vp, _vp]),
+    "moe_dispatch": (_int, [_vp, _i64, _int, _int, _int, _vp, _int, _int, _i64, _vp, _i64, _vp,
+                            _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _vp, _vp, _vp,
+                            _vp]),
     "moe_dispatch_permute_consume": (_int, [_vp, _int, _i64, _int, _i64, _vp, _i64, _vp, _int,
                                             _vp, _vp, _int, _vp, _vp, _vp, _i64, _vp, _vp, _i64,
                                             _vp, _vp]),
@@ -252,6 +255,52 @@ def moe_dispatch_permute(x: torch.Tensor, L: Layout, xp: Optional[torch.Tensor] 
         _stream(stream))
     _check(rc, "moe_dispatch_permute")
     return (xp, xp_scales) if dt == DTYPE_E4M3 else xp
+
+
+def moe_dispatch(topk_idx: torch.Tensor, x: torch.Tensor, E: int, R: int,
+                 layout: Optional[Layout] = None, xp: Optional[torch.Tensor] = None,
+                 x_scales: Optional[torch.Tensor] = None,
+                 xp_scales: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                 P_cap: Optional[int] = None, stream=None):
+    """moe_dispatch_layout followed by moe_dispatch_permute in one call (the
+    permute's first row loads overlap the layout).  Returns (layout, xp) or,
+    for E4M3 codes, (layout, xp, xp_scales)."""
+    _cuda(topk_idx, "topk_idx", torch.int32)
+    _cuda(x, "x", contiguous=False)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    T, K = topk_idx.shape
+    if x.shape[0] != T:
+        raise ValueError(f"x has {x.shape[0]} rows but topk_idx has {T}")
+    H = x.shape[1]
+    if x.dtype == torch.bfloat16:
+        dt, el = DTYPE_BF16, torch.bfloat16
+    elif x.dtype in (torch.uint8, torch.float8_e4m3fn):
+        dt, el = DTYPE_E4M3, x.dtype
+    else:
+        raise TypeError("x must be bfloat16 or E4M3 (uint8 / float8_e4m3fn)")
+    L = layout or alloc_layout(T, K, E, R, topk_idx.device, P_cap)
+    if L.workspace is None:
+        raise ValueError("this layout has no workspace")
+    if xp is None:
+        xp = torch.empty((L.P_cap, H), dtype=el, device=x.device)
+    _shape(_cuda(xp, "xp"), "xp", (L.P_cap, H))
+    xs_stride = 0
+    if dt == DTYPE_E4M3:
+        _cuda(x_scales, "x_scales", torch.float32, contiguous=False)
+        _shape(x_scales, "x_scales", (T, H // 128))
+        xs_stride = x_scales.stride(0)
+        if xp_scales is None:
+            xp_scales = torch.empty((L.P_cap, H // 128), dtype=torch.float32, device=x.device)
+        _shape(_cuda(xp_scales, "xp_scales", torch.float32), "xp_scales", (L.P_cap, H // 128))
+    rc = lib().moe_dispatch(
+        _ptr(topk_idx), T, K, E, R, _ptr(x), dt, H, x.stride(0), _ptr(x_scales), xs_stride,
+        _ptr(L.expert_counts), _ptr(L.expert_offsets), _ptr(L.rank_counts), _ptr(L.rank_offsets),
+        _ptr(L.dst_row), _ptr(L.row_src), _ptr(L.tile_ready), L.P_cap, _ptr(L.workspace),
+        L.workspace.numel(), _ptr(xp), _ptr(xp_scales), _ptr(L.work), _ptr(status),
+        _stream(stream))
+    _check(rc, "moe_dispatch")
+    return (L, xp, xp_scales) if dt == DTYPE_E4M3 else (L, xp)
 
 
 def moe_dispatch_permute_consume(x: torch.Tensor, L: Layout, xp: Optional[torch.Tensor] = None,

@@ -227,6 +227,27 @@ MOE_API int moe_dispatch_permute(const void* x, int dtype, int64_t T, int H, int
                          int32_t* d_status, void* stream);
 
 /*
+ * Dispatch in one call ([DEP] fused unzip; [ASC] expand_x, expand_idx,
+ * ep_send_counts): moe_dispatch_layout followed by moe_dispatch_permute, with
+ * the same arguments, outputs, errors and results as those two calls made
+ * back to back on `stream` (x, dtype, H, x_row_stride, x_scales,
+ * x_scales_row_stride, xp, xp_scales and work as in moe_dispatch_permute;
+ * the rest as in moe_dispatch_layout; counters are always maintained when
+ * tile_ready is given).  In one call the permute's first row loads overlap
+ * the layout, so x (and x_scales) must not overlap any buffer the call
+ * writes; like every input, x must be complete in stream order when the call
+ * is enqueued.  Every argument is checked before anything is launched.
+ */
+MOE_API int moe_dispatch(const int32_t* topk_idx, int64_t T, int K, int E, int R,
+                         const void* x, int dtype, int H, int64_t x_row_stride,
+                         const float* x_scales, int64_t x_scales_row_stride,
+                         int32_t* expert_counts, int32_t* expert_offsets, int32_t* rank_counts,
+                         int32_t* rank_offsets, int32_t* dst_row, int32_t* row_src,
+                         uint32_t* tile_ready, int64_t P_cap, void* workspace,
+                         size_t workspace_bytes, void* xp, float* xp_scales, uint32_t* work,
+                         int32_t* d_status, void* stream);
+
+/*
  * Counter-driven overlap: the dispatch permute and a consumer of its
  * chunk-completion counters in ONE cooperative launch ([DEP]: a consumer
  * acquires each chunk once and must then see all of it).  Warp 0 of every
