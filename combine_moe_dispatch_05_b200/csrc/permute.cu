@@ -21,12 +21,14 @@
 //     from a claim counter, so CTAs on faster SMs take more of it and all
 //     finish together (see the token-ordered pipeline below).
 //   * counters: a row's +1 is released only after its bulk-store group has
-//     completed (cp.async.bulk.wait_group), behind a proxy fence; releases
-//     are batched (one completion wait and one fence.acq_rel.gpu per 8
-//     groups, 4 groups behind) followed by relaxed adds (the pull request's
-//     atom.acq_rel.gpu on every add is a full fence per row).  FP8 scale
-//     rows are copied by the 32 lanes with plain stores before the same
-//     release.
+//     completed (cp.async.bulk.wait_group), behind a proxy fence and a
+//     fence.acq_rel.gpu, with relaxed adds (the pull request's
+//     atom.acq_rel.gpu on every add is a full fence per row).  Each CTA
+//     counts its rows per 128-row tile in a shared-memory table and adds
+//     the counts when all of its stores have completed, so no completion
+//     wait stalls the copy loop; with too many tiles for the table it
+//     releases in batches as it goes.  FP8 scale rows are copied by the 32
+//     lanes with plain stores before the same release.
 //   * the tile-ordered pipeline for the counter-driven overlap (at the end of
 //     this file) fills 16-row items in tile order and releases each as it
 //     lands.
@@ -91,6 +93,7 @@ struct PermArgs {
   int64_t pad_per_ticket;    // padding rows named by one padding ticket
   int first_tickets;         // tickets each CTA claims at once to fill its ring
   int early_x;               // issue the first batch's x loads before the grid wait
+  int tile_table;            // tiles counted per CTA and released once at its end (0: batched)
 };
 
 __device__ __forceinline__ uint32_t chunk_len(const PermArgs& a, int ch) {
@@ -127,6 +130,7 @@ __device__ __forceinline__ uint32_t chunk_len(const PermArgs& a, int ch) {
 constexpr int kRelBatch = MOE_PERM_REL_BATCH;
 constexpr int kTokRing = 64;  // tokens whose destination rows are held (until released)
 constexpr int kScRing = kMaxStages;  // tokens whose E4M3 scales are held (until processed)
+constexpr int64_t kMaxTableTiles = 8192;  // tile table of at most 16 KB per CTA
 constexpr int kRecRing = 64;  // committed bulk groups not yet released
 static_assert(kRecRing > kRelLag + kRelBatch && kTokRing > kMaxStages + kRelLag + kRelBatch,
               "rings too small for the release lag");
@@ -171,6 +175,9 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
   uint8_t* zero = smem + (size_t)S * a.stage_bytes;
   uint64_t* bar = reinterpret_cast<uint64_t*>(zero + a.stage_bytes);
   float* s_sc = reinterpret_cast<float*>(bar + kMaxStages);  // [kScRing][scale_cols] (E4M3)
+  // rows written per 128-row tile by this CTA (tile_table mode)
+  uint16_t* tbl = reinterpret_cast<uint16_t*>(s_sc + kScRing * a.scale_cols);
+  const bool table = a.tile_table > 0;
 
   const int64_t tpt = a.tokens_per_ticket;
   const int64_t n_tok = (a.T + tpt - 1) / tpt;  // token tickets
@@ -244,7 +251,8 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
   };
   // lane 0: release the groups older than the newest kRelLag once they completed
   auto retire = [&]() {
-    if (a.tile_ready == nullptr || n_commit - n_rel < (uint32_t)(kRelLag + kRelBatch)) return;
+    if (table || a.tile_ready == nullptr || n_commit - n_rel < (uint32_t)(kRelLag + kRelBatch))
+      return;
     bulk_wait_all<kRelLag>();
     fence_proxy_async_global();
     fence_acq_rel_gpu();
@@ -285,6 +293,16 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
     if (lane == 0) {
       bulk_commit();
       push_rec(kRecPad, qa, qb);
+      if (table) {
+        PadCursor tc;
+        tc.seek(sh.padpref, E, qa);
+        for (int64_t q = qa; q < qb;) {
+          const int64_t r = pad_row(tc, q);
+          const int64_t q_end = min(qb, (int64_t)sh.padpref[tc.e + 1]);
+          tbl[r / kTile] += (uint16_t)(q_end - q);
+          q = q_end;
+        }
+      }
       retire();
     }
   };
@@ -396,6 +414,9 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
   if (lane == 0) sh.padpref[E] = run;
   for (uint32_t i = lane * 16; i < a.stage_bytes; i += 32 * 16)
     *reinterpret_cast<uint4*>(zero + i) = make_uint4(0, 0, 0, 0);
+  if (table)
+    for (int i = lane * 8; i < a.tile_table; i += 32 * 8)
+      *reinterpret_cast<uint4*>(tbl + i) = make_uint4(0, 0, 0, 0);
   fence_proxy_async_shared();
   __syncwarp();
   if (__any_sync(0xffffffffu, bad) || (int64_t)sh.off[E] > a.P_cap || sh.off[0] != 0) {
@@ -451,6 +472,9 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
       bulk_commit();
       sh.stage_grp[s] = (int32_t)n_commit;
       push_rec(ch == nch - 1 ? kRecToken : kRecNone, j, 0);
+      if (table && ch == nch - 1)
+        for (int k = 0; k < K; ++k)
+          if (rows[k] >= 0) tbl[rows[k] / kTile] += 1;
       retire();
     }
     ++u;
@@ -468,7 +492,8 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
         if (!mbar_wait_bounded(&bar[v % S], (uint32_t)((v / S) & 1))) break;
     }
     bulk_wait_all<0>();
-    if (ok && a.tile_ready != nullptr && n_commit != n_rel) {
+    if (ok && table) fence_proxy_async_global();
+    if (ok && !table && a.tile_ready != nullptr && n_commit != n_rel) {
       fence_proxy_async_global();
       fence_acq_rel_gpu();
       while (n_rel != n_commit) {
@@ -483,8 +508,15 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
         ++n_rel;
       }
     }
-    finish_claims(a.work);  // the last CTA out returns both words to zero
   }
+  if (ok && table) {
+    // every row this CTA wrote has landed: one release per tile it touched
+    __syncwarp();
+    fence_acq_rel_gpu();
+    for (int i = lane; i < a.tile_table; i += 32)
+      if (tbl[i] != 0) atomic_add_relaxed_gpu(a.tile_ready + i, (uint32_t)tbl[i]);
+  }
+  if (lane == 0) finish_claims(a.work);  // the last CTA out returns both words to zero
 }
 
 __global__ void __launch_bounds__(32, 1) permute_kernel(const PermArgs a) {
@@ -924,7 +956,13 @@ int permute_launch(const void* x, int dtype, int64_t T, int H, int64_t x_row_str
   if (optin < 0) return MOE_ERR_CUDA;
   const int ctas_per_sm = perm_ctas_per_sm(a.row_bytes);
   const size_t scale_ring = (size_t)kScRing * a.scale_cols * sizeof(float);
-  const size_t dyn = size_ring(a, ctas_per_sm, sizeof(PermShared), optin, scale_ring);
+  // Per-CTA tile table (16-bit counts) when the tiles fit kMaxTableTiles;
+  // else releases in batches during the copy.
+  const int64_t n_tiles = (P_cap + kTile - 1) / kTile;
+  a.tile_table = (tile_ready != nullptr && n_tiles <= kMaxTableTiles)
+                     ? (int)((n_tiles + 7) / 8 * 8) : 0;
+  const size_t dyn = size_ring(a, ctas_per_sm, sizeof(PermShared), optin,
+                               scale_ring + (size_t)a.tile_table * sizeof(uint16_t));
   if (dyn == 0) return MOE_ERR_UNSUPPORTED;
   if (!allow_max_dyn_smem(permute_kernel, dev, optin, g_dyn_perm)) return MOE_ERR_CUDA;
 

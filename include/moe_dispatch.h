@@ -200,12 +200,15 @@ MOE_API int moe_dispatch_layout_static(const int32_t* topk_idx, int64_t T, int K
  * Out:
  *   xp        [P_cap, H] of `dtype`, contiguous, 16-byte aligned.
  *   xp_scales fp32 [P_cap, H/128] (E4M3 only; NULL for bf16).
- *   tile_ready (nullable) counters zeroed by the layout call; each finished
- *            row adds 1 to tile_ready[row/128] after its bytes (and scales)
- *            are globally visible, behind a gpu-scope release (a
- *            fence.acq_rel.gpu per group of rows, then relaxed atomic adds),
- *            so a tile whose counter reads 128 with an ld.acquire.gpu is
- *            complete.
+ *   tile_ready (nullable) counters zeroed by the layout call; every row
+ *            written adds 1 to tile_ready[row/128] once its bytes (and
+ *            scales) are globally visible, behind a gpu-scope release
+ *            (fence.acq_rel.gpu, then relaxed atomic adds), so a tile whose
+ *            counter reads 128 with an ld.acquire.gpu is complete.  Each
+ *            CTA counts its rows per tile and adds them when all of its rows
+ *            have landed (with more than 8192 tiles: in batches as it goes);
+ *            a tile's rows come from tokens across the whole batch, so tiles
+ *            complete near the end of the launch either way.
  * Scheduling words:
  *   work     device uint32 [2], 4-byte aligned, non-NULL: the claim counter
  *            through which the copy pipelines take tokens and padding rows as
