@@ -130,7 +130,7 @@ __device__ __forceinline__ uint32_t chunk_len(const PermArgs& a, int ch) {
 constexpr int kRelBatch = MOE_PERM_REL_BATCH;
 constexpr int kTokRing = 64;  // tokens whose destination rows are held (until released)
 constexpr int kScRing = kMaxStages;  // tokens whose E4M3 scales are held (until processed)
-constexpr int64_t kMaxTableTiles = 8192;  // tile table of at most 16 KB per CTA
+constexpr int64_t kMaxTableTiles = 8192;  // tile table of at most 8 KB per CTA
 constexpr int kRecRing = 64;  // committed bulk groups not yet released
 static_assert(kRecRing > kRelLag + kRelBatch && kTokRing > kMaxStages + kRelLag + kRelBatch,
               "rings too small for the release lag");
@@ -175,8 +175,8 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
   uint8_t* zero = smem + (size_t)S * a.stage_bytes;
   uint64_t* bar = reinterpret_cast<uint64_t*>(zero + a.stage_bytes);
   float* s_sc = reinterpret_cast<float*>(bar + kMaxStages);  // [kScRing][scale_cols] (E4M3)
-  // rows written per 128-row tile by this CTA (tile_table mode)
-  uint16_t* tbl = reinterpret_cast<uint16_t*>(s_sc + kScRing * a.scale_cols);
+  // rows written per 128-row tile by this CTA (tile_table mode; at most 128)
+  uint8_t* tbl = reinterpret_cast<uint8_t*>(s_sc + kScRing * a.scale_cols);
   const bool table = a.tile_table > 0;
 
   const int64_t tpt = a.tokens_per_ticket;
@@ -299,7 +299,7 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
         for (int64_t q = qa; q < qb;) {
           const int64_t r = pad_row(tc, q);
           const int64_t q_end = min(qb, (int64_t)sh.padpref[tc.e + 1]);
-          tbl[r / kTile] += (uint16_t)(q_end - q);
+          tbl[r / kTile] += (uint8_t)(q_end - q);
           q = q_end;
         }
       }
@@ -415,7 +415,7 @@ __device__ __forceinline__ void permute_warp(const PermArgs& a, uint8_t* smem, P
   for (uint32_t i = lane * 16; i < a.stage_bytes; i += 32 * 16)
     *reinterpret_cast<uint4*>(zero + i) = make_uint4(0, 0, 0, 0);
   if (table)
-    for (int i = lane * 8; i < a.tile_table; i += 32 * 8)
+    for (int i = lane * 16; i < a.tile_table; i += 32 * 16)
       *reinterpret_cast<uint4*>(tbl + i) = make_uint4(0, 0, 0, 0);
   fence_proxy_async_shared();
   __syncwarp();
@@ -956,13 +956,13 @@ int permute_launch(const void* x, int dtype, int64_t T, int H, int64_t x_row_str
   if (optin < 0) return MOE_ERR_CUDA;
   const int ctas_per_sm = perm_ctas_per_sm(a.row_bytes);
   const size_t scale_ring = (size_t)kScRing * a.scale_cols * sizeof(float);
-  // Per-CTA tile table (16-bit counts) when the tiles fit kMaxTableTiles;
-  // else releases in batches during the copy.
+  // Per-CTA tile table (one byte per tile) when the tiles fit
+  // kMaxTableTiles; else releases in batches during the copy.
   const int64_t n_tiles = (P_cap + kTile - 1) / kTile;
   a.tile_table = (tile_ready != nullptr && n_tiles <= kMaxTableTiles)
-                     ? (int)((n_tiles + 7) / 8 * 8) : 0;
+                     ? (int)((n_tiles + 15) / 16 * 16) : 0;
   const size_t dyn = size_ring(a, ctas_per_sm, sizeof(PermShared), optin,
-                               scale_ring + (size_t)a.tile_table * sizeof(uint16_t));
+                               scale_ring + (size_t)a.tile_table);
   if (dyn == 0) return MOE_ERR_UNSUPPORTED;
   if (!allow_max_dyn_smem(permute_kernel, dev, optin, g_dyn_perm)) return MOE_ERR_CUDA;
 
