@@ -112,3 +112,36 @@ def test_permute_kinds_share_one_pair_of_words_in_stream_order():
     rs = L.row_src[:P].long()
     real = rs >= 0
     assert torch.equal(a[:P][real], x[(rs[real] // s.K)])
+
+
+@pytest.mark.parametrize("H,fp8", [(8, False), (128, True)])
+def test_permute_with_more_tiles_than_the_table_releases_in_batches(H, fp8):
+    """T=131072, K=8, E=256: about 1.08 M padded rows, 8447 tiles, more than a
+    CTA's tile table holds, so the counters are released in batches during
+    the copy.  Bytes (and E4M3 scales) against the oracle, complete counters,
+    scheduling words back at zero."""
+    s = W.Spec("many_tiles", 131072, H, 256, 8, 8, "uniform", seed=404 + H)
+    ids = W.topk_ids(s)
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    assert (ref.P_cap + 127) // 128 > 8192
+    st = ops.new_status()
+    L = ops.moe_dispatch_layout(ids.to(DEV), s.E, s.R, status=st)
+    if fp8:
+        codes, xs = W.e4m3_codes(s), W.block_scales(s)
+        xp, xps = ops.moe_dispatch_permute(codes.to(DEV), L, x_scales=xs.to(DEV), status=st)
+        xp_ref = np.zeros((ref.P_cap, H), np.uint8)
+        xps_ref = np.zeros((ref.P_cap, H // 128), np.float32)
+        oracle.permute_rows(codes.numpy(), ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+        oracle.permute_rows(xs.numpy(), ref.dst_row, s.K, ref.counts, ref.offsets, xps_ref)
+    else:
+        x = W.tokens(s)
+        xp = ops.moe_dispatch_permute(x.to(DEV), L, status=st)
+        xp_ref = np.zeros((ref.P_cap, H), np.uint16)
+        oracle.permute_rows(W.as_u16(x), ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    assert _words_zero(L) and ops.read_status(st) == 0
+    P = ref.P
+    got = xp[:P].cpu().numpy() if fp8 else dev_u16(xp)[:P]
+    assert np.array_equal(got, xp_ref[:P])
+    if fp8:
+        assert np.array_equal(xps[:P].cpu().numpy().view(np.uint32), xps_ref[:P].view(np.uint32))
+    assert _counters_complete(L, P)
