@@ -2,7 +2,10 @@
 // the FP8 dispatch (codes travel with their per-block scales; DeepEP pull
 // request "Intra-node compute compensation ...", Testing: the FP8 dispatch
 // path).  s = amax / 448 in fp32 (1 when the block is all zero), codes =
-// E4M3(x / s) with IEEE fp32 division, round to nearest even, saturating.
+// E4M3(x / s) with the fp32 quotient rounded to nearest even (the IEEE
+// division's result, formed with one reciprocal per block and Markstein's
+// correction step: div8_by_scale), converted with round to nearest even,
+// saturating.
 //
 // A 256-thread CTA owns a token row (grid-stride over tokens): thread i holds
 // 16-byte vectors i, i+256, ... of the bf16 row, four at a time with all four
@@ -20,6 +23,38 @@ namespace {
 
 constexpr int kQThreads = 256;
 constexpr int kQU = 4;  // columns per thread per batch
+
+// x / s rounded to nearest even, for a divisor s shared by many x (one
+// 128-channel block's scale).  r must be the correctly rounded reciprocal
+// RN(1/s) (the __frcp_rn intrinsic), computed once per block.  Markstein's
+// theorem (P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990; also Muller et
+// al., Handbook of Floating-Point Arithmetic, the section on division with
+// an FMA): if r is within half an ulp of 1/s and q0 = RN(x*r) within one ulp
+// of x/s, then with the exact residual e = x - s*q0 (one FMA), RN(q0 + e*r)
+// is RN(x/s).  It needs the operands and the residual away from underflow,
+// which div8_by_scale arranges.  A zero residual returns q0 as it is, which
+// keeps the sign of a zero quotient.
+__device__ __forceinline__ float div_by_shared(float x, float s, float r) {
+  const float q0 = __fmul_rn(x, r);
+  const float e = __fmaf_rn(-q0, s, x);
+  return e == 0.0f ? q0 : __fmaf_rn(e, r, q0);
+}
+
+// The eight quotients f[k] / s of one 16-byte bf16 vector, each rounded to
+// nearest even as an IEEE division would round it, for a block scale
+// s = amax / 448 with |f[k]| <= amax.  A scale below 2^-100 is first
+// multiplied, with the f[k], by 2^64: exact (powers of two, no overflow since
+// |f| <= 448 s), and the quotients are unchanged.  Then s >= 2^-85, so every
+// quotient that an E4M3 code can tell apart (above 2^-24) has an operand,
+// product and residual in the normal range, where Markstein's step holds.
+__device__ __forceinline__ void div8_by_scale(const float* f, float s, float* out) {
+  const float m = s < 0x1p-100f ? 0x1p64f : 1.0f;
+  const float ss = __fmul_rn(s, m);
+  const float r = __frcp_rn(ss);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) out[k] = div_by_shared(__fmul_rn(f[k], m), ss, r);
+}
 
 __global__ void __launch_bounds__(kQThreads)
 quantize_e4m3_kernel(const uint16_t* __restrict__ x, int64_t T, int H, int64_t stride,
@@ -57,10 +92,12 @@ quantize_e4m3_kernel(const uint16_t* __restrict__ x, int64_t T, int H, int64_t s
         for (int o = 8; o > 0; o >>= 1)
           amax = fmaxf(amax, __shfl_xor_sync(half_mask, amax, o, 16));
         const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        float qf[8];
+        div8_by_scale(f, s, qf);
         uint32_t c[2] = {0u, 0u};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const float2 pr = make_float2(__fdiv_rn(f[2 * k], s), __fdiv_rn(f[2 * k + 1], s));
+          const float2 pr = make_float2(qf[2 * k], qf[2 * k + 1]);
           const uint32_t c2 = (uint32_t)__nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
           c[k >> 1] |= c2 << (16 * (k & 1));
         }

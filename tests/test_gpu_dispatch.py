@@ -283,6 +283,49 @@ def test_quantize_then_dispatch_fp8_pipeline():
     assert np.array_equal(xps.cpu().numpy()[:P], xps_ref[:P])
 
 
+def _extreme_block_rows(T, H, seed):
+    """bf16 rows whose 128-channel blocks span the whole bf16 range: each
+    block gets a random magnitude 2^m (m from -133, the smallest subnormal,
+    up to 127) times N(0,1) values, some blocks all zero, some single-value
+    blocks, some with values pushed to exact bf16 extremes."""
+    g = torch.Generator().manual_seed(seed)
+    nb = H // 128
+    mags = torch.randint(-133, 128, (T, nb, 1), generator=g).to(torch.float64)
+    x = torch.randn((T, nb, 128), generator=g, dtype=torch.float64) * torch.exp2(mags)
+    x = x.clamp(-3.0e38, 3.0e38)
+    zero = torch.rand((T, nb, 1), generator=g) < 0.05
+    x = torch.where(zero, torch.zeros_like(x), x)
+    one = torch.rand((T, nb, 1), generator=g) < 0.05
+    x = torch.where(one & (torch.arange(128) > 0), torch.zeros_like(x), x)
+    return x.view(T, H).to(torch.float32).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_quantize_e4m3_extreme_block_scales(seed):
+    """Block scales from bf16 subnormals (scale below 2^-100: the quotient
+    path rescales by 2^64 first) to near the largest bf16 values: codes and
+    scales bit for bit against the oracle, standalone and fused."""
+    T, H = 1024, 1024
+    x = _extreme_block_rows(T, H, seed)
+    q_ref, s_ref = oracle.quantize_e4m3(W.as_u16(x))
+    assert float(np.min(s_ref[s_ref > 0])) < 2.0 ** -100     # the tiny-scale path is used
+    q, qs = ops.moe_quantize_e4m3(x.to(DEV))
+    assert np.array_equal(qs.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    s = W.Spec("extreme", T, H, 16, 4, 4, "uniform", seed=seed)
+    ids = W.topk_ids(s)
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    L, _ = run_layout(ids, s.E, s.R)
+    xp, xps = ops.moe_dispatch_permute_quant(x.to(DEV), L)
+    xp_ref = np.zeros((ref.P_cap, H), np.uint8)
+    xps_ref = np.zeros((ref.P_cap, H // 128), np.float32)
+    oracle.permute_rows(q_ref, ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    oracle.permute_rows(s_ref, ref.dst_row, s.K, ref.counts, ref.offsets, xps_ref)
+    assert np.array_equal(xp.cpu().numpy()[:ref.P], xp_ref[:ref.P])
+    assert np.array_equal(xps.cpu().numpy()[:ref.P].view(np.uint32),
+                          xps_ref[:ref.P].view(np.uint32))
+
+
 def test_quantize_e4m3_round_trip_bound_on_gpu_codes():
     """Codes and scales from the GPU quantiser, decoded by torch's own E4M3
     conversion: |x - q*s| <= 2^-4 |x| where x/s is a normal E4M3 number and
