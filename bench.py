@@ -485,6 +485,15 @@ def run_ours(args, world, rank, local):
                                         t["layout_permute_then_consumer"], 3)}
         res["shared_expert_overlap"] = shared_expert_overlap(ops, torch, dev, flush, stream, ids,
                                                              sc, x, L, xp, E, R)
+        res["l2_writeback"] = l2_writeback(torch, dev, flush, stream, [
+            ("combine", lambda: ops.moe_combine(xp, L.dst_row, sc, out=out, status=st2)),
+            ("combine_bwd", lambda: ops.moe_combine_bwd(g, xp, sc, L, grad_y=gy, grad_scales=gs,
+                                                        status=st2)),
+            ("dispatch_bwd", lambda: ops.moe_dispatch_bwd(gy, L.dst_row, T, K, grad_x=gx,
+                                                          status=st2)),
+        ])
+        if ops.read_status(st2) != 0:
+            raise RuntimeError(f"device status {ops.read_status(st2)} in the L2 runs")
         res["other_workloads"] = extra_workloads(args, dev, flush, stream)
         res["planner"] = plan_on(L, E, R, ops)
 
@@ -646,6 +655,35 @@ def time_calls(torch, calls, flush, steps, stream):
             b.synchronize()
             ts.append(a.elapsed_time(b) * 1e3)
         out[name] = statistics.median(ts)
+    return out
+
+
+def l2_writeback(torch, dev, flush, stream, calls):
+    """Each gather kernel timed after two kinds of L2 flush: the standard one
+    (a 256 MiB write, which leaves L2 full of dirty lines that the kernel then
+    has to write back to HBM, as it would the previous layer's output) and the
+    same write followed by a 256 MiB read (L2 left holding clean lines).  The
+    difference is the write-back of what earlier work left in L2, traffic that
+    is not the kernel's own; every headline number keeps the standard flush."""
+    rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    acc = torch.empty((), dtype=torch.float32, device=dev)
+
+    class CleanFlush:
+        @staticmethod
+        def zero_():
+            flush.zero_()
+            torch.sum(rd, dim=0, out=acc)
+
+    dirty = time_calls(torch, calls, flush, 30, stream)
+    clean = time_calls(torch, calls, CleanFlush, 30, stream)
+    out = {"what": "medians of 30 launches after a 256 MiB write (dirty L2, the standard "
+                   "flush) and after the same write plus a 256 MiB read (clean L2). After the "
+                   "clean flush a kernel's own last writes (up to its output size, at most L2) "
+                   "also stay in L2 unpaid, so clean_us is a lower bound, not a throughput",
+}
+    for name, _ in calls:
+        out[name] = {"dirty_us": round(dirty[name], 1), "clean_us": round(clean[name], 1),
+                     "difference_us": round(dirty[name] - clean[name], 1)}
     return out
 
 
