@@ -326,6 +326,49 @@ def test_quantize_e4m3_extreme_block_scales(seed):
                           xps_ref[:ref.P].view(np.uint32))
 
 
+def _every_bf16_under(amax_bits):
+    """128-channel blocks led by the bf16 value amax_bits (which fixes the
+    block's scale), followed by every bf16 value of either sign whose
+    magnitude does not exceed it, 127 to a block (the last block padded with
+    zeros)."""
+    mags = np.arange(0, amax_bits + 1, dtype=np.uint16)
+    vals = np.concatenate([mags, mags[1:] | np.uint16(0x8000)])
+    n = (len(vals) + 126) // 127
+    rows = np.zeros((n, 128), np.uint16)
+    rows[:, 0] = amax_bits
+    body = np.zeros(n * 127, np.uint16)
+    body[:len(vals)] = vals
+    rows[:, 1:] = body.reshape(n, 127)
+    return rows
+
+
+def test_quantize_e4m3_every_bf16_value_under_inexact_scales():
+    """For block maxima whose scale amax/448 is inexact (and one whose scale
+    is below 2^-100, and a subnormal one), every bf16 value up to the block
+    maximum: the quotient x/s must round exactly as the IEEE division does,
+    so codes agree bit for bit with the oracle's, standalone and fused."""
+    amaxes = [0x3F80, 0x4040, 0x3DCD, 0x40B0, 0x43DF, 0x43E1, 0x7149, 0x1000, 0x0005]
+    x = W.from_u16(np.concatenate([_every_bf16_under(a) for a in amaxes]))
+    T, H = x.shape
+    q_ref, s_ref = oracle.quantize_e4m3(W.as_u16(x))
+    assert float(np.min(s_ref)) < 2.0 ** -100
+    q, qs = ops.moe_quantize_e4m3(x.to(DEV))
+    assert np.array_equal(qs.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    s = W.Spec("every_bf16", T, H, 16, 4, 4, "uniform", seed=7)
+    ids = W.topk_ids(s)
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    L, _ = run_layout(ids, s.E, s.R)
+    xp, xps = ops.moe_dispatch_permute_quant(x.to(DEV), L)
+    xp_ref = np.zeros((ref.P_cap, H), np.uint8)
+    xps_ref = np.zeros((ref.P_cap, H // 128), np.float32)
+    oracle.permute_rows(q_ref, ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    oracle.permute_rows(s_ref, ref.dst_row, s.K, ref.counts, ref.offsets, xps_ref)
+    assert np.array_equal(xp.cpu().numpy()[:ref.P], xp_ref[:ref.P])
+    assert np.array_equal(xps.cpu().numpy()[:ref.P].view(np.uint32),
+                          xps_ref[:ref.P].view(np.uint32))
+
+
 def test_quantize_e4m3_round_trip_bound_on_gpu_codes():
     """Codes and scales from the GPU quantiser, decoded by torch's own E4M3
     conversion: |x - q*s| <= 2^-4 |x| where x/s is a normal E4M3 number and
