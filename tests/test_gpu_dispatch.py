@@ -236,7 +236,7 @@ def test_permute_fp8_full_prefill_sampled_rows():
 
 # ---------------------------------------------------------- quantiser ----
 @pytest.mark.parametrize("T,H", [(64, 1024), (1000, 7168), (3, 128), (300, 384), (70, 8320),
-                                 (5, 20480)])
+                                 (5, 20480), (8192, 7168)])
 def test_quantize_e4m3_parity(T, H):
     s = W.config(3).with_(T=T, H=H)
     x = W.tokens(s)
