@@ -361,7 +361,8 @@ MOE_API int moe_dispatch_bwd(const void* grad_xp, const int32_t* dst_row, int64_
  *   q = E4M3(x / s) with fp32 division, round-to-nearest-even, saturating
  *       at +-448.
  * In:  x bf16 [T, H], row stride x_row_stride elements (multiple of 8),
- *      16-byte aligned; H % 128 == 0.
+ *      16-byte aligned (32-byte aligned x with a stride that is a multiple of
+ *      16 is read 32 bytes per load); H % 128 == 0.
  * Out: q uint8 [T, H] contiguous, 8-byte aligned (16-byte aligned q is
  *      written with 16-byte stores); q_scales fp32 [T, H/128] contiguous.
  */
