@@ -168,7 +168,10 @@ constexpr int kBwdThreads = MOE_BWD_THREADS;
 constexpr int kBwdWarps = kBwdThreads / 32;
 
 // resident CTAs per SM asked of the register allocator, per column batch
-constexpr int bwd_min_blocks(int u) { return u == 8 ? 3 : u == 1 ? 5 : 4; }
+constexpr int bwd_min_blocks(int u) { return u == 8 ? 3 : u == 2 ? 4 : 5; }
+// most slots a token can have for a column batch: the launch picks kU >= 2
+// only when K <= 8 / kU (gather_u), so the dot products need no more
+__host__ __device__ constexpr int bwd_max_k(int u) { return u == 1 ? MOE_MAX_TOPK : 8 / u; }
 
 template <int kU>
 __global__ void __launch_bounds__(kBwdThreads, bwd_min_blocks(kU))
@@ -210,9 +213,10 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
     fetch(t + gridDim.x, buf ^ 1);
     const int* rows = s_row[buf];
     const float* scs = s_sc[buf];
-    float dot[MOE_MAX_TOPK];
+    constexpr int kMaxK = bwd_max_k(kU);
+    float dot[kMaxK];
 #pragma unroll
-    for (int k = 0; k < MOE_MAX_TOPK; ++k) dot[k] = 0.0f;
+    for (int k = 0; k < kMaxK; ++k) dot[k] = 0.0f;
 
     for (int vb = tid; vb < V; vb += kBwdThreads * kU) {
       float gf[kU][8];
@@ -228,7 +232,7 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
         }
       }
 #pragma unroll
-      for (int kb = 0; kb < MOE_MAX_TOPK; kb += kKB) {
+      for (int kb = 0; kb < kMaxK; kb += kKB) {
         if (kb >= K) break;
         uint4 yv[kKB][kU];
 #pragma unroll
@@ -284,7 +288,7 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
 
     // fixed-order reduction of the K dot products over the CTA
 #pragma unroll
-    for (int k = 0; k < MOE_MAX_TOPK; ++k) {
+    for (int k = 0; k < kMaxK; ++k) {
       if (k >= K) break;
       float d = dot[k];
 #pragma unroll
