@@ -34,9 +34,13 @@ constexpr int kKBatch = 8;       // gathers issued before reducing
 #ifndef MOE_GATHER_CTA_THREADS
 #define MOE_GATHER_CTA_THREADS 256
 #endif
-// resident 256-thread CTAs per SM asked of the register allocator, per column
-// batch: 4 (64 registers) for one column, fewer as the batch holds more loads
-constexpr int gather_min_blocks(int u) { return u == 1 ? 4 : u == 2 ? 3 : u == 4 ? 2 : 1; }
+// resident 256-thread CTAs per SM asked of the register allocator, per
+// column and row batch: 4 (64 registers) for one column, fewer as the batch
+// holds more loads; a batch of fewer than kKBatch loads (few slots per
+// token) leaves registers for 4 CTAs up to two columns, 3 at four
+constexpr int gather_min_blocks(int u, int kb) {
+  return u * kb < kKBatch ? (u <= 2 ? 4 : 3) : u == 1 ? 4 : u == 2 ? 3 : u == 4 ? 2 : 1;
+}
 constexpr int kCtaThreads = MOE_GATHER_CTA_THREADS;
 
 // CTA-per-token reduction: threads 0..K-1 fetch the next token's row indices
@@ -44,15 +48,16 @@ constexpr int kCtaThreads = MOE_GATHER_CTA_THREADS;
 // shared memory), so index latency stays off the critical path.  Each thread
 // handles kU columns at a time and issues kU * min(K, 8 / kU) 16-byte gathers
 // before reducing, so about eight loads are in flight per thread whatever K
-// is (kU = 8 / K rounded down to a power of two).
-template <bool kScaled, bool kShared, int kU>
-__global__ void __launch_bounds__(kCtaThreads, gather_min_blocks(kU))
+// is (kU = 8 / K rounded down to a power of two).  A batch holds kKB rows:
+// 8 / kU, or fewer when the token has fewer slots (K rounded up to a power of
+// two), so that short tokens do not hold registers for rows they lack.
+template <bool kScaled, bool kShared, int kU, int kKB>
+__global__ void __launch_bounds__(kCtaThreads, gather_min_blocks(kU, kKB))
 gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ dst_row,
                          const float* __restrict__ scales, const uint16_t* __restrict__ shared,
                          int64_t T, int K, int H, int64_t P_cap, uint16_t* __restrict__ out,
                          int32_t* status) {
   pdl_begin();
-  constexpr int kKB = kKBatch / kU;  // rows per batch
   __shared__ int32_t s_row[2][MOE_MAX_TOPK];
   __shared__ float s_sc[2][MOE_MAX_TOPK];
   const int tid = threadIdx.x;
@@ -336,7 +341,8 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
   }
 }
 
-std::atomic<int> g_occ_comb[12][moe_host::kMaxCachedDevices];
+// occupancy cache per (caller, kU, kKB): caller * 16 + log2(kU) * 4 + log2(kKB)
+std::atomic<int> g_occ_comb[48][moe_host::kMaxCachedDevices];
 std::atomic<int> g_occ_bwd[4][moe_host::kMaxCachedDevices];
 
 // kU = columns per thread per batch: 8 / K rounded down to a power of two,
@@ -347,12 +353,15 @@ inline int gather_u(int K, int V, int threads) {
   return u;
 }
 
-template <bool kScaled, bool kShared, int kU>
-int launch_gather_u(int slot, const uint16_t* y, const int32_t* dst_row, const float* scales,
+constexpr int log2_small(int v) { return v >= 8 ? 3 : v >= 4 ? 2 : v >= 2 ? 1 : 0; }
+
+template <bool kScaled, bool kShared, int kU, int kKB>
+int launch_gather_u(int caller, const uint16_t* y, const int32_t* dst_row, const float* scales,
                     const uint16_t* shared, int64_t T, int K, int H, int64_t P_cap,
                     uint16_t* out, int32_t* status, cudaStream_t s) {
   const int dev = moe_host::current_device();
-  auto kern = gather_reduce_cta_kernel<kScaled, kShared, kU>;
+  auto kern = gather_reduce_cta_kernel<kScaled, kShared, kU, kKB>;
+  const int slot = caller * 16 + log2_small(kU) * 4 + log2_small(kKB);
   const int bps = moe_host::blocks_per_sm(kern, kCtaThreads, 0, dev, g_occ_comb[slot]);
   int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
   if (grid > T) grid = T;
@@ -361,23 +370,50 @@ int launch_gather_u(int slot, const uint16_t* y, const int32_t* dst_row, const f
                           shared, T, K, H, P_cap, out, status);
 }
 
+// the row batch: 8 / kU rows, or K rounded up to a power of two when smaller
+template <bool kScaled, bool kShared, int kU>
+int launch_gather_rows(int caller, const uint16_t* y, const int32_t* dst_row,
+                       const float* scales, const uint16_t* shared, int64_t T, int K, int H,
+                       int64_t P_cap, uint16_t* out, int32_t* status, cudaStream_t s) {
+  constexpr int kFull = kKBatch / kU;
+  int kb = 1;
+  while (kb < K && kb < kFull) kb <<= 1;
+  if constexpr (kFull >= 8) {
+    if (kb == 4)
+      return launch_gather_u<kScaled, kShared, kU, 4>(caller, y, dst_row, scales, shared, T, K, H,
+                                                      P_cap, out, status, s);
+  }
+  if constexpr (kFull >= 4) {
+    if (kb == 2)
+      return launch_gather_u<kScaled, kShared, kU, 2>(caller, y, dst_row, scales, shared, T, K, H,
+                                                      P_cap, out, status, s);
+  }
+  if constexpr (kFull >= 2) {
+    if (kb == 1)
+      return launch_gather_u<kScaled, kShared, kU, 1>(caller, y, dst_row, scales, shared, T, K, H,
+                                                      P_cap, out, status, s);
+  }
+  return launch_gather_u<kScaled, kShared, kU, kFull>(caller, y, dst_row, scales, shared, T, K, H,
+                                                      P_cap, out, status, s);
+}
+
 template <bool kScaled, bool kShared>
-int launch_gather(int slot, const uint16_t* y, const int32_t* dst_row, const float* scales,
+int launch_gather(int caller, const uint16_t* y, const int32_t* dst_row, const float* scales,
                   const uint16_t* shared, int64_t T, int K, int H, int64_t P_cap, uint16_t* out,
                   int32_t* status, cudaStream_t s) {
   switch (gather_u(K, H >> 3, kCtaThreads)) {
     case 8:
-      return launch_gather_u<kScaled, kShared, 8>(slot * 4 + 0, y, dst_row, scales, shared, T, K,
-                                                  H, P_cap, out, status, s);
+      return launch_gather_rows<kScaled, kShared, 8>(caller, y, dst_row, scales, shared, T, K, H,
+                                                     P_cap, out, status, s);
     case 4:
-      return launch_gather_u<kScaled, kShared, 4>(slot * 4 + 1, y, dst_row, scales, shared, T, K,
-                                                  H, P_cap, out, status, s);
+      return launch_gather_rows<kScaled, kShared, 4>(caller, y, dst_row, scales, shared, T, K, H,
+                                                     P_cap, out, status, s);
     case 2:
-      return launch_gather_u<kScaled, kShared, 2>(slot * 4 + 2, y, dst_row, scales, shared, T, K,
-                                                  H, P_cap, out, status, s);
+      return launch_gather_rows<kScaled, kShared, 2>(caller, y, dst_row, scales, shared, T, K, H,
+                                                     P_cap, out, status, s);
     default:
-      return launch_gather_u<kScaled, kShared, 1>(slot * 4 + 3, y, dst_row, scales, shared, T, K,
-                                                  H, P_cap, out, status, s);
+      return launch_gather_rows<kScaled, kShared, 1>(caller, y, dst_row, scales, shared, T, K, H,
+                                                     P_cap, out, status, s);
   }
 }
 
