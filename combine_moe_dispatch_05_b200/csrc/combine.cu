@@ -37,9 +37,9 @@ constexpr int kKBatch = 8;       // gathers issued before reducing
 // resident 256-thread CTAs per SM asked of the register allocator, per
 // column and row batch: 4 (64 registers) for one column, fewer as the batch
 // holds more loads; a batch of fewer than kKBatch loads (few slots per
-// token) leaves registers for 4 CTAs up to two columns, 3 at four
+// token) leaves registers for 4 CTAs up to two columns, 2 at four
 constexpr int gather_min_blocks(int u, int kb) {
-  return u * kb < kKBatch ? (u <= 2 ? 4 : 3) : u == 1 ? 4 : u == 2 ? 3 : u == 4 ? 2 : 1;
+  return u * kb < kKBatch ? (u <= 2 ? 4 : 2) : u == 1 ? 4 : u == 2 ? 3 : u == 4 ? 2 : 1;
 }
 constexpr int kCtaThreads = MOE_GATHER_CTA_THREADS;
 
@@ -49,8 +49,9 @@ constexpr int kCtaThreads = MOE_GATHER_CTA_THREADS;
 // handles kU columns at a time and issues kU * min(K, 8 / kU) 16-byte gathers
 // before reducing, so about eight loads are in flight per thread whatever K
 // is (kU = 8 / K rounded down to a power of two).  A batch holds kKB rows:
-// 8 / kU, or fewer when the token has fewer slots (K rounded up to a power of
-// two), so that short tokens do not hold registers for rows they lack.
+// 8 / kU, or fewer when the token has fewer slots (K itself with one column
+// per thread, K rounded up to a power of two with more), so that short
+// tokens do not hold registers for rows they lack.
 template <bool kScaled, bool kShared, int kU, int kKB>
 __global__ void __launch_bounds__(kCtaThreads, gather_min_blocks(kU, kKB))
 gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ dst_row,
@@ -84,6 +85,17 @@ gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restri
       for (int i = 0; i < kU; ++i)
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[i][e] = 0.0f;
+      // when the row batch leaves registers free, the shared term's vectors
+      // go out with the first batch of gathers (they are added after the k
+      // loop either way, as the definition orders them)
+      constexpr bool kEarlyShared = kShared && kU * kKB < kKBatch;
+      uint4 sv[kEarlyShared ? kU : 1];
+#pragma unroll
+      for (int i = 0; i < (kEarlyShared ? kU : 1); ++i) {
+        const int vec = vb + i * kCtaThreads;
+        sv[i] = (kEarlyShared && vec < V) ? ld_nc_v4(shared + t * H + (int64_t)vec * 8)
+                                          : make_uint4(0, 0, 0, 0);
+      }
       for (int kb = 0; kb < K; kb += kKB) {
         uint4 v[kKB][kU];
 #pragma unroll
@@ -124,8 +136,9 @@ gather_reduce_cta_kernel(const uint16_t* __restrict__ y, const int32_t* __restri
         const int vec = vb + i * kCtaThreads;
         if (vec >= V) continue;
         if (kShared) {
-          const uint4 sv = ld_nc_v4(shared + t * H + (int64_t)vec * 8);
-          const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
+          const uint4 sh = kEarlyShared ? sv[kEarlyShared ? i : 0]
+                                        : ld_nc_v4(shared + t * H + (int64_t)vec * 8);
+          const uint32_t w[4] = {sh.x, sh.y, sh.z, sh.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             acc[i][2 * q] = __fadd_rn(acc[i][2 * q], bf16_lo(w[q]));
@@ -341,8 +354,8 @@ combine_bwd_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ 
   }
 }
 
-// occupancy cache per (caller, kU, kKB): caller * 16 + log2(kU) * 4 + log2(kKB)
-std::atomic<int> g_occ_comb[48][moe_host::kMaxCachedDevices];
+// occupancy cache per (caller, kU, kKB): caller * 40 + log2(kU) * 10 + kKB
+std::atomic<int> g_occ_comb[120][moe_host::kMaxCachedDevices];
 std::atomic<int> g_occ_bwd[4][moe_host::kMaxCachedDevices];
 
 // kU = columns per thread per batch: 8 / K rounded down to a power of two,
@@ -361,7 +374,7 @@ int launch_gather_u(int caller, const uint16_t* y, const int32_t* dst_row, const
                     uint16_t* out, int32_t* status, cudaStream_t s) {
   const int dev = moe_host::current_device();
   auto kern = gather_reduce_cta_kernel<kScaled, kShared, kU, kKB>;
-  const int slot = caller * 16 + log2_small(kU) * 4 + log2_small(kKB);
+  const int slot = caller * 40 + log2_small(kU) * 10 + kKB;
   const int bps = moe_host::blocks_per_sm(kern, kCtaThreads, 0, dev, g_occ_comb[slot]);
   int64_t grid = (int64_t)moe_host::sm_count(dev) * bps;
   if (grid > T) grid = T;
@@ -370,12 +383,31 @@ int launch_gather_u(int caller, const uint16_t* y, const int32_t* dst_row, const
                           shared, T, K, H, P_cap, out, status);
 }
 
-// the row batch: 8 / kU rows, or K rounded up to a power of two when smaller
+// the row batch: 8 / kU rows, or fewer when K is smaller: K itself for one
+// column per thread, K rounded up to a power of two for more
 template <bool kScaled, bool kShared, int kU>
 int launch_gather_rows(int caller, const uint16_t* y, const int32_t* dst_row,
                        const float* scales, const uint16_t* shared, int64_t T, int K, int H,
                        int64_t P_cap, uint16_t* out, int32_t* status, cudaStream_t s) {
   constexpr int kFull = kKBatch / kU;
+  if constexpr (kU == 1) {
+    switch (K < kFull ? K : kFull) {
+      case 7:
+        return launch_gather_u<kScaled, kShared, 1, 7>(caller, y, dst_row, scales, shared, T, K,
+                                                       H, P_cap, out, status, s);
+      case 6:
+        return launch_gather_u<kScaled, kShared, 1, 6>(caller, y, dst_row, scales, shared, T, K,
+                                                       H, P_cap, out, status, s);
+      case 5:
+        return launch_gather_u<kScaled, kShared, 1, 5>(caller, y, dst_row, scales, shared, T, K,
+                                                       H, P_cap, out, status, s);
+      case 3:
+        return launch_gather_u<kScaled, kShared, 1, 3>(caller, y, dst_row, scales, shared, T, K,
+                                                       H, P_cap, out, status, s);
+      default:
+        break;  // 1, 2, 4 and 8 below
+    }
+  }
   int kb = 1;
   while (kb < K && kb < kFull) kb <<= 1;
   if constexpr (kFull >= 8) {
