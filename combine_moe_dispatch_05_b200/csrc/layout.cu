@@ -10,7 +10,8 @@
 // Two launches, deterministic by construction (positions come from ordered
 // scans, never from the order in which atomics arrive):
 //   1. count:  each 1024-thread block owns a contiguous run of whole tokens
-//      (<= 2048 slots).  Warp w walks its 64-slot segment 32 slots at a time;
+//      (<= 1024 slots up to 65536 slots in all, else <= 2048).  Warp w walks
+//      its 32- or 64-slot segment 32 slots at a time;
 //      ballots over the id bits group the lanes holding the same expert, the
 //      popcount of the lower lanes is the rank inside the group, and a
 //      per-warp 16-bit shared histogram carries the running count.  A scan
@@ -29,8 +30,11 @@ namespace {
 
 constexpr int kLayoutThreads = 1024;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
-constexpr int kSlotsPerBlock = 2048;
-constexpr int kItersPerWarp = kSlotsPerBlock / kLayoutThreads;  // 2 x 32 slots per warp
+// A block owns kIters x 1024 slots (kIters 32-slot steps per warp): 1024 when
+// the batch has at most kSmallLayoutSlots slots, where more, shorter blocks
+// finish sooner; 2048 above, where the assign kernel's column sums over the
+// per-block totals would grow with the block count instead.
+constexpr int64_t kSmallLayoutSlots = 65536;
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -111,6 +115,7 @@ __device__ __forceinline__ void fill_words(uint32_t* dst, int64_t n, uint32_t va
   if (gt < n - tail0) dst[tail0 + gt] = value;
 }
 
+template <int kIters>
 __global__ void __launch_bounds__(kLayoutThreads)
 layout_count_kernel(const int32_t* __restrict__ ids, int64_t T, int K, int E,
                     int tokens_per_block, int32_t* __restrict__ block_counts,
@@ -120,7 +125,7 @@ layout_count_kernel(const int32_t* __restrict__ ids, int64_t T, int K, int E,
   pdl_begin();
   if (trigger) pdl_trigger();
   __shared__ __align__(16) uint16_t hist[kLayoutWarps * MOE_MAX_EXPERTS];  // [warp][E]
-  __shared__ int32_t s_ids[kSlotsPerBlock];
+  __shared__ int32_t s_ids[kIters * kLayoutThreads];
 
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
@@ -149,12 +154,12 @@ layout_count_kernel(const int32_t* __restrict__ ids, int64_t T, int K, int E,
 
   const int warp = tid >> 5, lane = tid & 31;
   uint16_t* my_hist = hist + warp * Es;
-  int my_e[kItersPerWarp], my_r[kItersPerWarp];
+  int my_e[kIters], my_r[kIters];
   int err = 0;
   const int nbits = id_bits(E);
 #pragma unroll
-  for (int it = 0; it < kItersPerWarp; ++it) {
-    const int rel = warp * (kItersPerWarp * 32) + it * 32 + lane;
+  for (int it = 0; it < kIters; ++it) {
+    const int rel = warp * (kIters * 32) + it * 32 + lane;
     count_step(rel, n_b, rel < n_b ? s_ids[rel] : -1, K, E, nbits, s_ids, my_hist, lane, err,
                my_e[it], my_r[it]);
   }
@@ -175,12 +180,13 @@ layout_count_kernel(const int32_t* __restrict__ ids, int64_t T, int K, int E,
   __syncthreads();
 
 #pragma unroll
-  for (int it = 0; it < kItersPerWarp; ++it) {
-    const int rel = warp * (kItersPerWarp * 32) + it * 32 + lane;
+  for (int it = 0; it < kIters; ++it) {
+    const int rel = warp * (kIters * 32) + it * 32 + lane;
     if (rel < n_b) slot_rank[s0 + rel] = my_e[it] >= 0 ? my_hist[my_e[it]] + my_r[it] : -1;
   }
 }
 
+template <int kIters>
 __global__ void __launch_bounds__(kLayoutThreads)
 layout_assign_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ slot_rank,
                      const int32_t* __restrict__ block_counts, int nb, int64_t T, int K, int E,
@@ -206,9 +212,9 @@ layout_assign_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict_
   const int nt = (int)max((int64_t)0, min((int64_t)tokens_per_block, T - t0));
   const int n_b = nt * K;
   const int64_t s0 = t0 * K;
-  int my_rank[kItersPerWarp], my_id[kItersPerWarp];
+  int my_rank[kIters], my_id[kIters];
 #pragma unroll
-  for (int it = 0; it < kItersPerWarp; ++it) {
+  for (int it = 0; it < kIters; ++it) {
     const int i = tid + it * kLayoutThreads;
     my_rank[it] = i < n_b ? slot_rank[s0 + i] : -1;
     my_id[it] = i < n_b ? __ldg(ids + s0 + i) : 0;
@@ -279,7 +285,7 @@ layout_assign_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict_
 
   // 3. rows of this block's slots
 #pragma unroll
-  for (int it = 0; it < kItersPerWarp; ++it) {
+  for (int it = 0; it < kIters; ++it) {
     const int i = tid + it * kLayoutThreads;
     if (i >= n_b) continue;
     const int64_t slot = s0 + i;
@@ -300,7 +306,10 @@ layout_assign_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict_
   }
 }
 
-inline int tokens_per_block_for(int K) { return kSlotsPerBlock / K; }
+inline int layout_iters(int64_t T, int K) { return T * K <= kSmallLayoutSlots ? 1 : 2; }
+inline int tokens_per_block_for(int64_t T, int K) {
+  return layout_iters(T, K) * kLayoutThreads / K;
+}
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -309,7 +318,7 @@ inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 extern "C" size_t moe_layout_workspace_bytes(int64_t T, int K, int E) {
   if (T < 0 || K < 1 || K > MOE_MAX_TOPK || E < 1 || E > MOE_MAX_EXPERTS) return (size_t)-1;
-  const int tpb = moe::tokens_per_block_for(K);
+  const int tpb = moe::tokens_per_block_for(T, K);
   const int64_t nb = T > 0 ? (T + tpb - 1) / tpb : 1;
   return moe::align256((size_t)nb * E * sizeof(int32_t)) +
          moe::align256((size_t)(T > 0 ? T : 1) * K * sizeof(int32_t));
@@ -344,20 +353,22 @@ int layout_launch(const int32_t* topk_idx, int64_t T, int K, int E, int R,
   if (dry_run) return MOE_OK;
 
   const int64_t n_tiles = (P_cap + kTile - 1) / kTile;
-  const int tpb = tokens_per_block_for(K);
+  const int tpb = tokens_per_block_for(T, K);
   const int nb = T > 0 ? (int)((T + tpb - 1) / tpb) : 1;
   int32_t* block_counts = static_cast<int32_t*>(workspace);
   int32_t* slot_rank = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
                                                   align256((size_t)nb * E * sizeof(int32_t)));
 
-  int st = moe_host::launch(layout_count_kernel, dim3(nb), dim3(kLayoutThreads), 0, s, topk_idx, T,
-                            K, E, tpb, block_counts, slot_rank, row_src, P_cap, tile_ready,
-                            n_tiles, d_status, trigger);
+  const bool small = layout_iters(T, K) == 1;
+  int st = moe_host::launch(small ? layout_count_kernel<1> : layout_count_kernel<2>, dim3(nb),
+                            dim3(kLayoutThreads), 0, s, topk_idx, T, K, E, tpb, block_counts,
+                            slot_rank, row_src, P_cap, tile_ready, n_tiles, d_status, trigger);
   if (st != MOE_OK) return st;
-  return moe_host::launch(layout_assign_kernel, dim3(nb), dim3(kLayoutThreads), 0, s, topk_idx,
-                          (const int32_t*)slot_rank, (const int32_t*)block_counts, nb, T, K, E, R,
-                          tpb, expert_counts, expert_offsets, rank_counts, rank_offsets, dst_row,
-                          row_src, P_cap, d_status, trigger);
+  return moe_host::launch(small ? layout_assign_kernel<1> : layout_assign_kernel<2>, dim3(nb),
+                          dim3(kLayoutThreads), 0, s, topk_idx, (const int32_t*)slot_rank,
+                          (const int32_t*)block_counts, nb, T, K, E, R, tpb, expert_counts,
+                          expert_offsets, rank_counts, rank_offsets, dst_row, row_src, P_cap,
+                          d_status, trigger);
 }
 }  // namespace moe
 

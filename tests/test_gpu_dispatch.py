@@ -64,7 +64,12 @@ def test_layout_parity_hot_expert_everywhere():
     (1000, 16, 512, 512), (3000, 1, 2, 2), (129, 2, 3, 1), (257, 7, 64, 16), (4097, 6, 64, 16),
     # runs of 2048 slots per block: exact multiples and one token past them
     (4096, 8, 256, 8), (4097, 8, 256, 8), (2048, 16, 512, 8), (2049, 16, 64, 4),
-    (10912, 3, 9, 3), (10913, 3, 9, 3), (700, 5, 40, 8), (3000, 7, 100, 4)])
+    (10912, 3, 9, 3), (10913, 3, 9, 3), (700, 5, 40, 8), (3000, 7, 100, 4),
+    # runs of 1024 slots per block (batches of at most 65536 slots), and both
+    # sides of that bound
+    (128, 8, 256, 8), (129, 8, 256, 8), (1024, 1, 2, 2), (1025, 1, 2, 2), (341, 3, 9, 3),
+    (342, 3, 9, 3), (8192, 8, 256, 8), (8193, 8, 256, 8), (21845, 3, 9, 3),
+    (21846, 3, 9, 3), (65536, 1, 4, 2), (65537, 1, 4, 2)])
 def test_layout_parity_edge_shapes(T, K, E, R):
     s = W.Spec("edge", T, 8, E, K, R, "uniform", seed=77 + T + K + E)
     ids = W.topk_ids(s) if T else torch.zeros((0, K), dtype=torch.int32)
