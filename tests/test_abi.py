@@ -48,6 +48,24 @@ def test_host_only_entry_points():
     assert ops.status_string(ops.ERR_TIMEOUT) == "device-side wait timed out"
 
 
+def test_layout_workspace_follows_the_block_size():
+    """The layout scratch holds per-block expert counts (one int32 per expert
+    per block) and one int32 rank per slot, each region padded to 256 bytes.
+    Blocks own 1024 slots when the batch has at most 65536, 2048 above."""
+    B.build()
+
+    def expect(T, K, E):
+        per_block = (1024 if T * K <= 65536 else 2048) // K  # whole tokens per block
+        nb = (T + per_block - 1) // per_block if T else 1
+        pad = lambda n: (n + 255) // 256 * 256
+        return pad(nb * E * 4) + pad(max(T, 1) * K * 4)
+
+    for T, K, E in [(4096, 8, 256), (8192, 8, 256), (8193, 8, 256), (21845, 3, 9),
+                    (21846, 3, 9), (65536, 1, 4), (65537, 1, 4), (32768, 8, 256), (1, 16, 512),
+                    (0, 4, 8), (116480, 8, 256)]:
+        assert ops.layout_workspace_bytes(T, K, E) == expect(T, K, E), (T, K, E)
+
+
 def test_host_argument_errors_launch_nothing():
     """Argument checks return before any CUDA call, so they run without a GPU."""
     B.build()
