@@ -48,6 +48,29 @@ def test_host_only_entry_points():
     assert ops.status_string(ops.ERR_TIMEOUT) == "device-side wait timed out"
 
 
+def test_dispatch_in_one_call_checks_both_halves_before_launching():
+    """moe_dispatch checks the layout's and the permute's arguments before it
+    launches either kernel: a bad permute argument returns its own code, not
+    a launch failure of the layout (there is no GPU here, so any launch would
+    return ERR_CUDA)."""
+    B.build()
+    L = ops.lib()
+    f = ctypes.c_void_p(256)
+    T, K, E, R, H = 4, 2, 4, 2, 64
+    ws = ops.layout_workspace_bytes(T, K, E)
+
+    def call(E=E, R=R, dtype=0, stride=H, P_cap=1024, work=f, ws_bytes=ws):
+        return L.moe_dispatch(f, T, K, E, R, f, dtype, H, stride, None, 0, f, f, f, f, f, f, f,
+                              P_cap, f, ws_bytes, f, None, work, None, None)
+
+    assert call(E=6, R=4) == ops.ERR_INVALID_ARG           # E % R != 0 (layout)
+    assert call(P_cap=128) == ops.ERR_CAPACITY             # P_cap below the bound (layout)
+    assert call(ws_bytes=ws - 4) == ops.ERR_INVALID_ARG    # workspace too small (layout)
+    assert call(dtype=7) == ops.ERR_UNSUPPORTED            # unknown dtype (permute)
+    assert call(stride=H - 8) == ops.ERR_INVALID_ARG       # row stride below H (permute)
+    assert call(work=None) == ops.ERR_INVALID_ARG          # no scheduling words (permute)
+
+
 def test_layout_workspace_follows_the_block_size():
     """The layout scratch holds per-block expert counts (one int32 per expert
     per block) and one int32 rank per slot, each region padded to 256 bytes.
