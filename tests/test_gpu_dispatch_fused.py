@@ -136,3 +136,36 @@ def test_dispatch_in_one_call_in_cuda_graph():
         assert int(L.work.abs().sum().item()) == 0
     assert ops.read_status(st) == 0
     del graph
+
+
+@pytest.mark.parametrize("kind", ["range", "duplicate"])
+def test_dispatch_in_one_call_reports_bad_ids(kind):
+    """Ids out of range or repeated inside a token: the status carries the
+    oracle's error, the layout and the expert-major buffer equal the
+    oracle's (an out-of-range slot takes no row; a repeated id is placed
+    twice), and the scheduling words are back at zero."""
+    s = W.config(4).with_(H=256)
+    ids = W.topk_ids(s).clone()
+    if kind == "range":
+        ids[100, 2] = s.E
+        ids[2000, 0] = -3
+        expect = oracle.ERR_EXPERT_RANGE
+    else:
+        ids[555, 1] = ids[555, 0]
+        expect = oracle.ERR_DUPLICATE_EXPERT
+    ref = oracle.layout(ids.numpy(), s.E, s.R)
+    assert ref.status == expect
+    x = W.tokens(s)
+    st = ops.new_status()
+    L = ops.alloc_layout(s.T, s.K, s.E, s.R, DEV)
+    xp = torch.zeros((L.P_cap, s.H), dtype=torch.bfloat16, device=DEV)
+    xp.view(torch.int16).fill_(SENT)
+    ops.moe_dispatch(ids.to(DEV), x.to(DEV), s.E, s.R, layout=L, xp=xp, status=st)
+    assert ops.read_status(st) == expect
+    assert np.array_equal(L.dst_row.cpu().numpy(), ref.dst_row)
+    assert np.array_equal(L.row_src.cpu().numpy()[:ref.P_cap], ref.row_src)
+    assert np.array_equal(L.expert_offsets.cpu().numpy(), ref.offsets)
+    xp_ref = np.full((ref.P_cap, s.H), SENT, np.uint16)
+    oracle.permute_rows(W.as_u16(x), ref.dst_row, s.K, ref.counts, ref.offsets, xp_ref)
+    assert np.array_equal(dev_u16(xp), xp_ref)
+    assert int(L.work.abs().sum().item()) == 0
